@@ -1,0 +1,254 @@
+"""Pins for the oracle's whole path (no GPU).
+
+Each test fixes the oracle against something other than itself: the FP64
+fold identity of the SmoothQuant section, the special cases the method
+reduces to (k = 0 is a plain MXFP4 GEMM, k = d_in a bfloat16 GEMM, s = 1
+leaves X untouched), a brute-force check of the top-k definition, the
+monotonicity of rounding that lets the score be read from act_scale, and
+error bounds against the unquantised product.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import w4a4_oracle as orc
+
+
+def _bf16_np(t: torch.Tensor) -> np.ndarray:
+    return t.float().numpy()
+
+
+def _small(T=64, d_in=96, d_out=48, seed=0, n_out=4):
+    spec = synth.XSpec("student3", 0.3, n_out, 8.0, 30.0)
+    X = _bf16_np(synth.gen_x(spec, T, d_in, seed))
+    W = _bf16_np(synth.gen_w(synth.WSpec(0.02), d_out, d_in, seed + 1))
+    return X, W
+
+
+@pytest.mark.parametrize("alpha", [0.5, 0.7])
+def test_fold_identity_fp64(alpha):
+    """(X ⊘ s)(s ⊙ W) = XW in exact arithmetic (W4A4 review §3.2, fold equation)."""
+    X, W = _small()
+    act = orc.col_absmax(X)
+    wsc = orc.col_absmax(W)
+    s32, _ = orc.smoothing_factors(act, wsc, alpha)
+    s = s32.astype(np.float64)
+    lhs = orc.smooth_activation(X.astype(np.float64), 1.0 / s) @ orc.fold_weight(W.astype(np.float64), s).T
+    rhs = X.astype(np.float64) @ W.astype(np.float64).T
+    rel = np.abs(lhs - rhs).max() / np.abs(rhs).max()
+    assert rel <= 1e-12
+
+
+def test_fold_axis_matters():
+    X, W = _small(d_in=64, d_out=64)
+    s, inv_s = orc.smoothing_factors(orc.col_absmax(X), orc.col_absmax(W), 0.5)
+    s = s.astype(np.float64)
+    good = orc.smooth_activation(X.astype(np.float64), 1 / s) @ orc.fold_weight(W.astype(np.float64), s).T
+    wrong = orc.smooth_activation(X.astype(np.float64), 1 / s) @ (W.astype(np.float64) * s[:, None]).T
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    assert np.abs(good - ref).max() < 1e-9 * np.abs(ref).max()
+    assert np.abs(wrong - ref).max() > 1e-3 * np.abs(ref).max()
+
+
+def test_smoothing_closed_forms():
+    # alpha = 0.5, a = 16, w = 1 -> s = 4 ; a = 1, w = 0.25 -> s = 1 / 0.5 = 2
+    s, inv_s = orc.smoothing_factors(np.array([16.0, 1.0], np.float32),
+                                     np.array([1.0, 0.25], np.float32), 0.5)
+    np.testing.assert_array_equal(s, [4.0, 2.0])
+    np.testing.assert_array_equal(inv_s, [0.25, 0.5])
+    # alpha = 0.7, a = 2^10, w = 2^-10 -> s = 2^7 * 2^3 = 2^10
+    s, _ = orc.smoothing_factors(np.array([1024.0], np.float32), np.array([2.0**-10], np.float32), 0.7)
+    assert abs(float(s[0]) - 1024.0) <= 1024.0 * 2**-22
+    # zero magnitudes are clamped at 1e-5: a = 0, w = 0, alpha = 0.5 -> s = 1e-5^0.5 / 1e-5^0.5 = 1
+    s, _ = orc.smoothing_factors(np.zeros(1, np.float32), np.zeros(1, np.float32), 0.5)
+    assert s[0] == 1.0
+
+
+def test_smoothing_balances_ranges_at_half():
+    """At alpha = 0.5 the smoothed activation channel max equals the folded
+    weight channel max (both are sqrt(a_j w_j)), the balance SmoothQuant targets."""
+    X, W = _small(T=128, d_in=64, d_out=64)
+    act, wsc = orc.col_absmax(X), orc.col_absmax(W)
+    s, inv_s = orc.smoothing_factors(act, wsc, 0.5)
+    xs = orc.col_absmax(orc.smooth_activation(X.astype(np.float64), 1.0 / s.astype(np.float64)))
+    ws = orc.col_absmax(orc.fold_weight(W.astype(np.float64), s.astype(np.float64)))
+    np.testing.assert_allclose(xs, ws, rtol=1e-6)
+    np.testing.assert_allclose(xs, np.sqrt(act.astype(np.float64) * wsc), rtol=1e-6)
+
+
+def test_score_equals_scaled_act_scale():
+    """max_t fl32(|x| * inv_s) = fl32(max_t |x| * inv_s): rounding is monotone,
+    so the score needs no second pass over X."""
+    X, W = _small(T=300, d_in=160)
+    act = orc.col_absmax(X)
+    _, inv_s = orc.smoothing_factors(act, orc.col_absmax(W), 0.6)
+    direct = orc.outlier_scores(X, inv_s)
+    shortcut = (act * inv_s).astype(np.float32)
+    np.testing.assert_array_equal(direct, shortcut)
+
+
+def test_topk_definition_brute_force():
+    rng = np.random.default_rng(1)
+    for trial in range(40):
+        d = int(rng.integers(1, 40))
+        score = rng.integers(0, 6, d).astype(np.float32)   # many ties on purpose
+        k = int(rng.integers(0, d + 1))
+        O, J = orc.select_outliers(score, k)
+        assert len(O) == k and len(J) == d - k
+        assert np.all(np.diff(O) > 0) and np.all(np.diff(J) > 0)
+        assert sorted(np.concatenate([O, J]).tolist()) == list(range(d))
+        for j in O:
+            for i in J:
+                assert score[j] > score[i] or (score[j] == score[i] and j < i)
+
+
+def test_topk_edges():
+    sc = np.array([1, 3, 3, 2], np.float32)
+    O, J = orc.select_outliers(sc, 0)
+    assert O.size == 0 and J.tolist() == [0, 1, 2, 3]
+    O, J = orc.select_outliers(sc, 1)
+    assert O.tolist() == [1] and J.tolist() == [0, 2, 3]
+    O, J = orc.select_outliers(sc, 4)
+    assert O.tolist() == [0, 1, 2, 3] and J.size == 0
+    with pytest.raises(ValueError):
+        orc.select_outliers(sc, 5)
+
+
+def test_identity_smoothing_is_plain_mxfp4():
+    """s = 1: prep quantises X itself; the O columns are copied unchanged."""
+    X, _ = _small(T=40, d_in=80)
+    O = np.array([3, 17, 40], np.int32)
+    J = np.setdiff1d(np.arange(80), O).astype(np.int32)
+    pa = orc.prep_activation(X, np.ones(80, np.float32), O, J)
+    np.testing.assert_array_equal(orc.bf16_bits_to_f32(pa["xo"]), X[:, O])
+    nb = orc.n_blocks(len(J))
+    XJ = np.zeros((40, nb * 32), np.float32)
+    XJ[:, :len(J)] = X[:, J]
+    sc, codes = orc.mxfp4_quantize_blocks(XJ.reshape(40, nb, 32))
+    np.testing.assert_array_equal(pa["sfa"], sc)
+    np.testing.assert_array_equal(pa["aq"], orc.pack_nibbles(codes.reshape(40, -1)))
+
+
+def test_k0_is_plain_mx_gemm_and_bounded():
+    """k = 0: the second branch vanishes; Y is the FP64 product of the
+    dequantised operands, and it stays within the element-wise quantisation
+    error bound of XW."""
+    X, W = _small(T=32, d_in=64, d_out=16)
+    Y, p = orc.linear_reference(X, W, 0.5, 0)
+    assert p["xo"].shape[1] == 0 and p["w_hp"].shape[1] == 0
+    A = orc.dequant_mxfp4(p["aq"], p["sfa"])
+    B = orc.dequant_mxfp4(p["wq"], p["sfb"])
+    np.testing.assert_array_equal(Y, A @ B.T)
+    # bound from the quantiser definition: |deq(v) - v| <= 2^e * (half spacing or saturation)
+    Vx = orc.smooth_activation(X.astype(np.float32), p["inv_s"]).astype(np.float64)
+    Vw = orc.fold_weight(W.astype(np.float32), p["s"]).astype(np.float64)
+
+    def err_bound(V, sf):
+        e = np.repeat(sf.astype(np.float64) - 127, 32, axis=1)[:, :V.shape[1]]
+        q = np.abs(V) * 2.0 ** -e
+        half = np.where(q < 2, 0.25, np.where(q < 4, 0.5, np.where(q <= 6, 1.0, q - 6)))
+        return half * 2.0 ** e
+
+    ex, ew = err_bound(Vx, p["sfa"]), err_bound(Vw, p["sfb"])
+    bound = (ex @ np.abs(Vw).T + np.abs(Vx) @ ew.T + ex @ ew.T) * (1 + 1e-6)
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    # Vx Vw^T differs from XW only by the fl32 roundings of the smoothing (2^-23 relative)
+    slack = 4 * 2.0**-23 * (np.abs(X.astype(np.float64)) @ np.abs(W.astype(np.float64)).T)
+    assert np.all(np.abs(Y - exact) <= bound + slack)
+
+
+def test_k_equals_din_is_bf16_gemm():
+    """k = d_in: no column is quantised; Y is the product of the bf16-rounded
+    smoothed operands and stays within bf16 rounding of XW."""
+    X, W = _small(T=24, d_in=48, d_out=20)
+    Y, p = orc.linear_reference(X, W, 0.7, 48)
+    assert p["aq"].shape[1] == 0 and p["xo"].shape[1] == 48
+    XO = orc.bf16_bits_to_f32(p["xo"]).astype(np.float64)
+    WO = orc.bf16_bits_to_f32(p["w_hp"]).astype(np.float64)
+    np.testing.assert_array_equal(Y, XO @ WO.T)
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    mag = np.abs(X.astype(np.float64)) @ np.abs(W.astype(np.float64)).T
+    # each operand: bf16 rounding (unit roundoff 2^-8: 8 significant bits)
+    # plus the fl32 roundings of the product and of inv_s
+    eps = 2.0**-8 + 2 * 2.0**-23
+    assert np.all(np.abs(Y - exact) <= (2 * eps + eps * eps) * mag * (1 + 1e-9))
+
+
+def test_split_sum_recombines():
+    """Y = X_J W_J + X_O W_O: with quantisation replaced by the identity the two
+    branches add up to the full product.  Checked by brute force: the oracle's
+    O/J split of columns, the compaction and the gathered bf16 columns index the
+    same channels on both operands."""
+    X, W = _small(T=16, d_in=70, d_out=12)
+    Y, p = orc.linear_reference(X, W, 0.5, 9)
+    O, J = p["O"], p["J"]
+    XO = orc.bf16_bits_to_f32(p["xo"]).astype(np.float64)
+    WO = orc.bf16_bits_to_f32(p["w_hp"]).astype(np.float64)
+    Vx = orc.smooth_activation(X.astype(np.float32), p["inv_s"])
+    Vw = orc.fold_weight(W.astype(np.float32), p["s"])
+    for t in range(4):
+        for n in range(4):
+            o_branch = sum(float(XO[t, i]) * float(WO[n, i]) for i in range(len(O)))
+            o_direct = sum(float(orc.bf16_bits_to_f32(orc.f32_to_bf16_bits(Vx[t, j:j + 1]))[0]) *
+                           float(orc.bf16_bits_to_f32(orc.f32_to_bf16_bits(Vw[n, j:j + 1]))[0])
+                           for j in O)
+            assert abs(o_branch - o_direct) <= 1e-12 * (1 + abs(o_direct))
+    A = orc.dequant_mxfp4(p["aq"], p["sfa"])
+    B = orc.dequant_mxfp4(p["wq"], p["sfb"])
+    j_branch = A @ B.T
+    np.testing.assert_allclose(Y, j_branch + XO @ WO.T, rtol=0, atol=1e-12)
+    # the J-branch, compacted, covers exactly the J channels: dequantised values
+    # stay within the quantisation error of the smoothed J columns
+    assert np.all(np.abs(A[:, :len(J)] - Vx[:, J]) <= np.abs(Vx[:, J]).max() * 0.5 + 1e-30)
+
+
+def test_32x32_tiles_share_one_scale():
+    X, W = _small(T=8, d_in=256, d_out=80)
+    _, p = orc.linear_reference(X, W, 0.5, 5, layout=orc.LAYOUT_32x32)
+    sfb = p["sfb"]
+    for g in range(0, 80, 32):
+        tile = sfb[g:g + 32]
+        assert np.all(tile == tile[0:1])
+    # the tile scale is the one of the tile's largest element
+    Vw = orc.fold_weight(W.astype(np.float32), p["s"])[:, p["J"]]
+    nb = sfb.shape[1]
+    VJ = np.zeros((80, nb * 32), np.float32)
+    VJ[:, :Vw.shape[1]] = Vw
+    amax = np.abs(VJ[0:32, 0:32]).max()
+    assert int(sfb[0, 0]) == int(orc.mx_shared_exponent(np.array([amax]))[0]) + 127
+
+
+def test_tiny_generator_matches_pages_statistics():
+    """The tiny workload's planted channels exceed 6.0, weights stay below 0.6
+    (review §3.1), and after smoothing the planted channels are the top-8."""
+    L = synth.TINY
+    X, W = synth.gen_layer(L)
+    X, W = _bf16_np(X), _bf16_np(W)
+    planted = synth.outlier_columns(L.x, L.d_in, L.seed).numpy()
+    act = orc.col_absmax(X)
+    assert np.all(act[planted] > 6.0)
+    assert orc.col_absmax(W).max() < 0.6
+    c = orc.calibrate(X, W, L.alpha, L.k)
+    assert sorted(c["O"].tolist()) == sorted(planted.tolist())
+
+
+def test_smoothing_and_splitting_help():
+    """Qualitative ordering stated in review §3.5: smoothing + splitting gives
+    a better SNR than plain W4A4 rounding on heavy-tailed activations."""
+    spec = synth.XSpec("student3", 0.3, 8, 8.0, 30.0)
+    X = _bf16_np(synth.gen_x(spec, 256, 512, 0))
+    W = _bf16_np(synth.gen_w(synth.WSpec(0.02), 128, 512, 1))
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+
+    def snr(Y):
+        return 10 * np.log10((exact**2).sum() / ((Y - exact)**2).sum())
+
+    O0 = np.zeros(0, np.int32)
+    J0 = np.arange(512, dtype=np.int32)
+    s1 = np.ones(512, np.float32)
+    pw = orc.pack_weight(W, s1, O0, J0)
+    pa = orc.prep_activation(X, s1, O0, J0)
+    plain = orc.dual_branch_product(pa["aq"], pa["sfa"], pa["xo"], pw["wq"], pw["sfb"], pw["w_hp"])
+    ours, _ = orc.linear_reference(X, W, 0.5, 8)
+    assert snr(ours) > snr(plain)

@@ -1,0 +1,477 @@
+"""Benchmark of the W4A4 dual-branch linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full|ffn0|ffn2|tiny|sweep]
+                    [--impl reference]
+
+One step is one pass of the whole path over one batch of synthetic input,
+for every layer of the workload: calibration absmax of X and of W, the
+finalisation (s, score, top-k), the weight pack, the activation prep and the
+dual-branch GEMM -- all through the C-ABI of libw4a4.  The default workload
+is the 720x1280x61 token count (T = 57600) through the FFN up-projection
+(5120 -> 13824, k = 32) and then the down-projection (13824 -> 5120, k = 64).
+
+``value`` is whole-step effective TFLOPS, 2 T d_in d_out summed over the
+layers divided by the step time (outlier columns counted at the 4-bit
+rate).  Per-kernel numbers come from CUDA events recorded on the launching
+stream around each launch inside the timed region.  Inputs are larger than
+L2 (X is 590 MB / 1.59 GB), so no flush is needed between steps.
+
+Under torchrun each rank runs the same per-GPU workload on its own token
+shard (weak scaling, no collective on the data path); the step time is the
+max over ranks, ``value`` counts the work of all ranks.
+
+``--impl reference`` times the CPU oracle (the numpy reference the tests
+check the GPU against) on a bounded row sample of the same workload, on
+rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dual-branch W4A4 GEMM TFLOPS & % of FP4 peak; prep kernel HBM GB/s"
+FP4_NOMINAL_TFLOPS = 9000.0        # B200 dense FP4, datasheet
+FP4_PER_BF16 = 4.0                 # nominal dense FP4 : BF16 ratio (9 / 2.25 PFLOP/s)
+HBM_NOMINAL_GBS = 8000.0
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host only; covered by gloo tests on CPU)
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(backend: str, world: int, rank: int, timeout_s: float = 120.0):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, world_size=world, rank=rank,
+                                timeout=datetime.timedelta(seconds=timeout_s))
+    return world > 1
+
+
+def dist_barrier(active: bool, device=None):
+    import torch.distributed as dist
+    if active:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def dist_max(value: float, active: bool, device) -> float:
+    """Max of a float over ranks (every rank calls it)."""
+    if not active:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, world: int, step_s_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return per_rank_units * world / step_s_max
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                smax.append(float(p[1]))
+                power.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def layer_bytes_prep(L, d) -> float:
+    """Algorithmic bytes of the prep kernel: X read + codes, scales and X_O written."""
+    return L.T * (2.0 * L.d_in + d.kj_pad / 2 + d.nblk + 2.0 * d.k_pad)
+
+
+class LayerRun:
+    """Device buffers and the C-ABI call sequence of one layer."""
+
+    def __init__(self, L, device, w4, synth):
+        import torch
+        self.L = L
+        self.w4 = w4
+        self.X, self.W = synth.gen_layer(L, device)
+        self.pw = w4.alloc_packed(L.d_in, L.d_out, L.k, L.layout, device)
+        self.act = w4.alloc_act(L.T, self.pw)
+        self.Y = torch.empty((L.T, L.d_out), dtype=torch.bfloat16, device=device)
+        self.d = self.pw.dims
+        self.launches = 0
+
+    def offline(self, ev=None):
+        """Calibration (absmax of X and W), finalisation and packing."""
+        w4, L, pw = self.w4, self.L, self.pw
+        if ev is not None:
+            ev[0].record()
+        w4.calib_observe(self.X, pw.act_scale, reset=True)
+        w4.calib_observe(self.W, pw.w_scale, reset=True)
+        if ev is not None:
+            ev[1].record()
+        w4.calib_finalize(pw.act_scale, pw.w_scale, L.alpha, L.k, pw.s, pw.inv_s, pw.score,
+                          pw.O if L.k else None, pw.jmap if L.k < L.d_in else None)
+        w4.pack_weight(self.W, pw)
+        return 2 + 2 + (1 if self.d.kj else 0) + (1 if L.k else 0)
+
+    def online(self, ev=None):
+        w4 = self.w4
+        if ev is not None:
+            ev[0].record()
+        w4.prep_act(self.X, self.pw, self.act)
+        if ev is not None:
+            ev[1].record()
+        w4.gemm_dual(self.act, self.L.T, self.pw, self.Y)
+        if ev is not None:
+            ev[2].record()
+        return 2
+
+
+def run_gpu(args):
+    import torch
+
+    import synth
+    import w4a4_mxfp4_outlier_b200 as w4
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    active = dist_init("nccl", world, rank)
+    layers = [L.with_(seed=L.seed + 1000 * rank) for L in synth.WORKLOADS[args.workload]]
+    runs = [LayerRun(L, device, w4, synth) for L in layers]
+    torch.cuda.synchronize()
+
+    def step(evs=None):
+        n = 0
+        for i, r in enumerate(runs):
+            n += r.offline(None if evs is None else evs[i]["off"])
+            n += r.online(None if evs is None else evs[i]["on"])
+        return n
+
+    for _ in range(args.warmup):
+        step()
+    st, bits = w4.last_error()
+    if st != w4.OK:
+        raise RuntimeError(f"device error word {bits:#x} during warm-up")
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[{"off": [mk(), mk()], "on": [mk(), mk(), mk()]} for _ in runs] for _ in range(args.steps)]
+    t0, t1 = mk(), mk()
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    dist_barrier(active, device)
+    clocks.start()
+    time.sleep(0.3)
+    t0.record()
+    launches = 0
+    for k in range(args.steps):
+        launches += step(evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    dist_barrier(active, device)
+    st, bits = w4.last_error()
+    if st != w4.OK:
+        raise RuntimeError(f"device error word {bits:#x} in the timed region")
+
+    step_ms = t0.elapsed_time(t1) / args.steps
+    step_ms_max = dist_max(step_ms, active, device)
+    flops = sum(L.flops for L in layers)
+    value = aggregate(flops, world, step_ms_max * 1e-3) / 1e12
+
+    gemm_ms = [sum(e[i]["on"][1].elapsed_time(e[i]["on"][2]) for e in evs) / args.steps
+               for i in range(len(runs))]
+    prep_ms = [sum(e[i]["on"][0].elapsed_time(e[i]["on"][1]) for e in evs) / args.steps
+               for i in range(len(runs))]
+    calib_ms = [sum(e[i]["off"][0].elapsed_time(e[i]["off"][1]) for e in evs) / args.steps
+                for i in range(len(runs))]
+    gemm_tflops = flops / (sum(gemm_ms) * 1e-3) / 1e12
+    prep_bytes = sum(layer_bytes_prep(r.L, r.d) for r in runs)
+    prep_gbs = prep_bytes / (sum(prep_ms) * 1e-3) / 1e9
+    calib_bytes = sum(2.0 * (r.L.T * r.L.d_in + r.L.d_out * r.L.d_in) for r in runs)
+    calib_gbs = calib_bytes / (sum(calib_ms) * 1e-3) / 1e9
+    online_tflops = flops / ((sum(gemm_ms) + sum(prep_ms)) * 1e-3) / 1e12
+
+    peaks, src = measured_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    roof = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+            "traffic": None,
+            "kernel": "gemm_dual_kernel",
+            "peak_source": f"{src}: bf16_tflops_sustained x {FP4_PER_BF16:g} (nominal FP4:BF16)",
+            "frac_of_nominal_fp4_9pf": round(gemm_tflops / FP4_NOMINAL_TFLOPS, 4)}
+
+    e2e = run_e2e(args, runs, w4, device, active) if not args.no_e2e else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(layers, runs)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
+            "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
+            "config": {"workload": f"{args.workload}: " + ", ".join(
+                f"{L.name} T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
+                f"{'32x32' if L.layout else '32x1'}" for L in layers),
+                "tokens_per_gpu": layers[0].T, "parallelism": f"token shards x{world}",
+                "l2": "inputs larger than L2 (no flush)",
+                "step": "calib absmax X,W + finalize + pack + prep + dual GEMM per layer"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clock_info,
+            "kernels": {
+                "gemm_ms": [round(x, 4) for x in gemm_ms],
+                "gemm_tflops": round(gemm_tflops, 1),
+                "prep_ms": [round(x, 4) for x in prep_ms],
+                "prep_gbs": round(prep_gbs, 1),
+                "prep_frac_hbm_measured": round(prep_gbs / peaks["hbm_gbs"], 4),
+                "prep_frac_hbm_nominal_8tbs": round(prep_gbs / HBM_NOMINAL_GBS, 4),
+                "calib_absmax_ms": [round(x, 4) for x in calib_ms],
+                "calib_absmax_gbs": round(calib_bytes / (sum(calib_ms) * 1e-3) / 1e9, 1),
+                "online_tflops": round(online_tflops, 1),
+            },
+        }
+        print(json.dumps(out), flush=True)
+    if active:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, runs, w4, device, active):
+    """Same step through the public calls with host buffers: every step copies
+    X and W from pinned host memory, runs the whole path and copies Y back."""
+    import torch
+    hosts = []
+    for r in runs:
+        hosts.append((r.X.cpu().pin_memory(), r.W.cpu().pin_memory(),
+                      torch.empty(r.Y.shape, dtype=r.Y.dtype).pin_memory()))
+    h2d = sum(x.numel() * 2 + w.numel() * 2 for x, w, _ in hosts)
+    d2h = sum(y.numel() * 2 for _, _, y in hosts)
+    steps = max(1, min(args.steps, 3))
+
+    def step():
+        for r, (xh, wh, yh) in zip(runs, hosts):
+            r.X.copy_(xh, non_blocking=True)
+            r.W.copy_(wh, non_blocking=True)
+            r.offline()
+            r.online()
+            yh.copy_(r.Y, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dist_barrier(active, device)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = dist_max(t0.elapsed_time(t1) / steps, active, device)
+    world = dist_env()[0]
+    flops = sum(r.L.flops for r in runs)
+    return {"value": round(aggregate(flops, world, ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+            "ms_per_step": round(ms, 3), "steps": steps,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(layers, rows_per_layer=64, out_per_layer=256, X_rows=None, W_rows=None):
+    """Run the oracle's whole path on a row sample of each layer.
+
+    Calibration sees the sampled rows, the pack covers `out_per_layer` output
+    channels, prep and the product the sampled tokens.  Returns (effective
+    FLOPs of the sample, seconds)."""
+    import numpy as np
+
+    from oracle import w4a4_oracle as orc
+    flops, secs = 0.0, 0.0
+    for i, L in enumerate(layers):
+        X = X_rows[i]
+        W = W_rows[i]
+        t = time.perf_counter()
+        c = orc.calibrate(X, W, L.alpha, L.k)
+        pw = orc.pack_weight(W, c["s"], c["O"], c["J"], L.layout)
+        pa = orc.prep_activation(X, c["inv_s"], c["O"], c["J"])
+        Y = orc.dual_branch_product(pa["aq"], pa["sfa"], pa["xo"], pw["wq"], pw["sfb"], pw["w_hp"])
+        secs += time.perf_counter() - t
+        flops += 2.0 * X.shape[0] * L.d_in * W.shape[0]
+        assert np.isfinite(Y).all()
+    return flops, secs
+
+
+def _host_samples(layers, runs=None, rows=64, outs=256):
+    import torch
+
+    import synth
+    Xs, Ws = [], []
+    for i, L in enumerate(layers):
+        if runs is not None:
+            X, W = runs[i].X, runs[i].W
+        else:
+            X = synth.gen_x(L.x, min(L.T, 2048), L.d_in, L.seed)
+            W = synth.gen_w(L.w, min(L.d_out, 2048), L.d_in, L.seed + 1)
+        idx = synth.sample_rows(X.shape[0], rows)
+        Xs.append(X[idx.to(X.device)].float().cpu().numpy())
+        Ws.append(W[:outs].float().cpu().numpy())
+    _ = torch
+    return Xs, Ws
+
+
+def cpu_baseline(layers, runs=None, rows=64, outs=256):
+    Xs, Ws = _host_samples(layers, runs, rows, outs)
+    flops, secs = oracle_sample(layers, rows, outs, Xs, Ws)
+    return {"value": round(flops / secs / 1e12, 8), "unit": "TFLOPS", "cores": _threads_used(),
+            "kind": "oracle",
+            "sample": f"{rows} token rows x {outs} output channels per layer, whole path "
+                      f"(calibrate, pack, prep, product) in numpy; {secs:.1f} s"}
+
+
+def run_reference(args):
+    import synth
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    layers = list(synth.WORKLOADS[args.workload])
+    Xs, Ws = _host_samples(layers, None, 64, 256)
+    for _ in range(args.warmup):
+        oracle_sample(layers, 64, 256, Xs, Ws)
+    tot_f, tot_s = 0.0, 0.0
+    for _ in range(args.steps):
+        f, s = oracle_sample(layers, 64, 256, Xs, Ws)
+        tot_f += f
+        tot_s += s
+    v = tot_f / tot_s / 1e12
+    cores = _threads_used()
+    sample = ("64 token rows x 256 output channels per layer of the workload, whole path "
+              "(calibrate, pack, prep, product) in the numpy oracle")
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 8), "unit": "TFLOPS",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(tot_s / args.steps * 1e3, 2), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (numpy oracle)",
+           "data": "synthetic", "config": {"workload": args.workload},
+           "cpu_baseline": {"value": round(v, 8), "unit": "TFLOPS", "cores": cores,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(v, 8), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="full", choices=["full", "ffn0", "ffn2", "tiny", "sweep"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)      # at least three untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * libw4a4 -- W4A4 dual-branch linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method (paper review "W4A4 Quantization for Inference on
+ * Wan2.2-I2V-A14B (ICME 2026 Challenge)", sections 3.2-3.4):
+ *
+ *   s_j  = act_scale_j^alpha / weight_scale_j^(1-alpha)          (sec. 3.2, eq. s_j)
+ *   Y    = (X / s)(s * W)                                          (sec. 3.2, fold eq.)
+ *   score_j = max_t |x_tj| on the smoothed X; O = top-k columns    (sec. 3.3, eq. score_j)
+ *   Y    = X_J W^(q)_J + X_O W^(hp)_O                              (sec. 3.3, eq. Y)
+ *
+ * with the J branch in MXFP4 (OCP E2M1 elements, one E8M0 scale per 32
+ * K-elements, shared exponent floor(log2 amax) - 2, round-half-to-even,
+ * saturation at +-6) and the O branch in bfloat16.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers owned by the caller unless a parameter
+ *    says "host".  The library never allocates device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream unless stated.
+ *  - Matrices are row-major.  X is [T, d_in] bf16 with row stride ldx
+ *    elements; W is [d_out, d_in] bf16 (row n = output channel n; this is the
+ *    transpose of the pages' d_in x d_out W); Y is [T, d_out] bf16.
+ *  - Arguments are validated before anything is launched.  On a non-OK
+ *    return nothing was enqueued and outputs are untouched.
+ *  - Supported shapes: d_in % 8 == 0, d_out % 16 == 0, row strides % 8 == 0,
+ *    all pointers 16-byte aligned, kj_pad <= 31744 (see w4a4_dims).
+ *    Anything else returns W4A4_ERR_UNSUPPORTED_SHAPE.
+ *  - Device-side failures (a pipeline wait that runs out, about 2 s) are
+ *    recorded in a device error word; w4a4_last_error() reads it.  No kernel
+ *    traps.
+ */
+#ifndef W4A4_H
+#define W4A4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4A4_ABI_VERSION 1
+
+typedef enum w4a4_status {
+  W4A4_OK = 0,
+  W4A4_ERR_INVALID_ARG = 1,      /* null pointer, negative size, alpha outside (0,1), k > d_in */
+  W4A4_ERR_UNSUPPORTED_SHAPE = 2,/* alignment or size outside the supported set above */
+  W4A4_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
+  W4A4_ERR_TIMEOUT = 4           /* a device pipeline wait ran out (see w4a4_last_error) */
+} w4a4_status;
+
+/* Weight scale layouts of the block packing (review sec. 3.4: "32x32 tiles"
+ * and K-major stripes; the stripe is 32x1 here, the MXFP4 block length). */
+typedef enum w4a4_wlayout {
+  W4A4_SF_32x1_KMAJOR = 0,  /* one E8M0 per 32 consecutive compacted K of one output row */
+  W4A4_SF_32x32_TILE = 1    /* one E8M0 per 32 output rows x 32 compacted K, stored on each row */
+} w4a4_wlayout;
+
+int w4a4_abi_version(void);
+const char* w4a4_status_string(w4a4_status s);
+
+/* ------------------------------------------------------------------------
+ * Geometry.  kj = d_in - k columns go to the 4-bit branch after compaction
+ * (O columns removed, review sec. 3.3); they are padded with zeros to kj_pad
+ * = round_up(kj, 256) so the GEMM runs whole 256-element K tiles.  nblk =
+ * kj_pad / 32 MX blocks per row.  k_pad = round_up(k, 16) bf16 columns per
+ * row of X_O and W_hp (zero padded).  sfa_rows(T) = round_up(T, 128);
+ * sfb_rows = round_up(d_out, 256).
+ *
+ * Scale-factor buffers use the block-scaled MMA layout: 512-byte atoms of
+ * 128 rows x 4 blocks, atoms ordered K-fastest; inside an atom row r, block
+ * b sits at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).  The byte of
+ * (row r, block b) is therefore
+ *   ((r / 128) * (nblk / 4) + b / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4.
+ * ------------------------------------------------------------------------ */
+typedef struct w4a4_dims {
+  int64_t d_in, d_out, k;
+  int64_t kj;       /* d_in - k */
+  int64_t kj_pad;   /* round_up(kj, 256) */
+  int64_t nblk;     /* kj_pad / 32 */
+  int64_t k_pad;    /* round_up(k, 16) */
+  int64_t sfb_rows; /* round_up(d_out, 256) */
+} w4a4_dims;
+
+/* Fills *out.  INVALID_ARG if out is NULL, a size is negative or k > d_in. */
+w4a4_status w4a4_get_dims(int64_t d_in, int64_t d_out, int64_t k, w4a4_dims* out);
+
+/* ------------------------------------------------------------------------
+ * Calibration (offline).  Review sec. 3.1-3.2: per-channel magnitudes of
+ * activations and weights; read here as the per-column absolute maximum.
+ * ------------------------------------------------------------------------ */
+
+/* absmax[j] = max(absmax[j], max_r |A[r, j]|) for j < cols (absmax zeroed
+ * first when reset != 0).  A: bf16 [rows, cols] with row stride lda.  Used
+ * for activation batches X [T, d_in] (act_scale) and for W [d_out, d_in]
+ * (weight_scale).  absmax: float32 [cols].  rows may be 0.  NaN inputs make
+ * the column NaN. */
+w4a4_status w4a4_calib_observe(const void* A, int64_t rows, int64_t cols, int64_t lda,
+                               float* absmax, int reset, void* stream);
+
+/* From act_scale and w_scale (float32 [d_in]) compute, on the device:
+ *   s[j]     = fl32( max(a,1e-5)^alpha / max(w,1e-5)^(1-alpha) )  in float64
+ *   inv_s[j] = fl32( 1 / s[j] )
+ *   score[j] = fl32( act_scale[j] * inv_s[j] )  (= max_t |fl32(x_tj inv_s_j)|,
+ *              the score on the smoothed activations; review sec. 3.3, 3.5)
+ *   O        = the k columns of largest score, ties to the lower index,
+ *              ascending (int32 [k]);  jmap = the other d_in - k columns
+ *              ascending (int32 [d_in - k]).
+ * Requires 0 < alpha < 1, 0 <= k <= d_in, 1 <= d_in <= 65535.  O may be NULL
+ * when k == 0 and jmap may be NULL when k == d_in. */
+w4a4_status w4a4_calib_finalize(const float* act_scale, const float* w_scale, int64_t d_in,
+                                double alpha, int64_t k, float* s, float* inv_s, float* score,
+                                int32_t* O, int32_t* jmap, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packed weight (offline).  Review sec. 3.2 (fold s into W), 3.3 (drop the O
+ * channels into the bf16 branch, static O kept as a sparse index list), 3.4
+ * (block-wise 4-bit packing with the exponent stored beside the payload).
+ * ------------------------------------------------------------------------ */
+typedef struct w4a4_weight_bytes {
+  size_t wq;    /* d_out * kj_pad / 2           E2M1 codes, row n: kj_pad/2 bytes */
+  size_t sfb;   /* sfb_rows * nblk               E8M0 codes, MMA layout            */
+  size_t w_hp;  /* d_out * k_pad * 2             bf16                              */
+} w4a4_weight_bytes;
+
+w4a4_status w4a4_weight_sizes(int64_t d_in, int64_t d_out, int64_t k, w4a4_weight_bytes* out);
+
+/* The per-layer record the online path reads.  All pointers are caller-owned
+ * device memory; the record itself lives on the host and is only read. */
+typedef struct w4a4_packed_weight {
+  int64_t d_in, d_out, k;
+  int32_t layout;        /* w4a4_wlayout */
+  int32_t reserved;
+  uint8_t* wq;           /* [d_out, kj_pad/2]: code of folded W[n, jmap[p]] at p (low nibble = even p) */
+  uint8_t* sfb;          /* MMA layout, sfb_rows x nblk; rows >= d_out hold code 0 */
+  void* w_hp;            /* bf16 [d_out, k_pad]: bf16_rn(fl32(W[n, O[i]] * s[O[i]])) */
+  const float* inv_s;    /* float32 [d_in] from w4a4_calib_finalize */
+  const int32_t* O;      /* int32 [k] ascending (NULL if k == 0) */
+  const int32_t* jmap;   /* int32 [d_in - k] ascending (NULL if k == d_in) */
+} w4a4_packed_weight;
+
+/* Fold and pack.  W: bf16 [d_out, d_in] with row stride ldw.  s, O, jmap from
+ * w4a4_calib_finalize.  Fills pw->wq, pw->sfb, pw->w_hp (which must point to
+ * buffers of the sizes w4a4_weight_sizes reports) and reads pw->d_in,
+ * d_out, k, layout.  Every element of wq/sfb/w_hp, padding included, is
+ * written.  Row n, compacted position p: v = fl32(W[n, jmap[p]] * s[jmap[p]]);
+ * MX blocks are p = 32b .. 32b+31 (zeros beyond kj). */
+w4a4_status w4a4_pack_weight(const void* W, int64_t ldw, const float* s,
+                             const w4a4_packed_weight* pw, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Online path.  Review sec. 3.2 (activations divided by s, then quantised)
+ * and sec. 3.3 (dual-branch GEMM).
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace w4a4_linear needs for T tokens: Aq
+ * (T * kj_pad / 2), SFA (round_up(T,128) * nblk) and X_O (T * k_pad * 2),
+ * each 1024-byte aligned. */
+w4a4_status w4a4_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int64_t k, size_t* bytes);
+
+/* Activation preparation (one pass over X).  For row t and column j,
+ * v = fl32(X[t, j] * inv_s[j]) (one IEEE multiply).  Writes
+ *   xo  bf16 [T, k_pad]       xo[t, i] = bf16_rn(v at j = O[i]), zeros for i >= k
+ *   aq  u8   [T, kj_pad/2]    E2M1 codes of v at j = jmap[p] (zeros for p >= kj)
+ *   sfa u8   MMA layout, round_up(T,128) x nblk; rows >= T are not written
+ * Each 32-element block takes e = clamp(floor(log2 amax) - 2, -127, 127),
+ * code = e + 127 (0 for an all-zero block), elements v * 2^-e rounded to
+ * E2M1 (nearest, ties to even, saturating at 6, sign kept).
+ * aq, sfa, xo may be NULL when their size is zero. */
+w4a4_status w4a4_prep_act(const void* X, int64_t T, int64_t ldx, const w4a4_packed_weight* pw,
+                          uint8_t* aq, uint8_t* sfa, void* xo, void* stream);
+
+/* Dual-branch product Y[t, n] = sum_p deq(aq)[t,p] deq(wq)[n,p]
+ *                              + sum_i xo[t,i] w_hp[n,i]
+ * accumulated in float32 in tensor memory (tcgen05 kind::mxf4 block-scaled
+ * tiles and kind::f16 tiles into the same accumulator), rounded to bf16.
+ * Y: bf16 [T, d_out] with row stride ldy. */
+w4a4_status w4a4_gemm_dual(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                           const w4a4_packed_weight* pw, void* Y, int64_t ldy, void* stream);
+
+/* The online layer: w4a4_prep_act into the workspace, then w4a4_gemm_dual.
+ * ws_bytes must be at least w4a4_workspace_size(T, ...). */
+w4a4_status w4a4_linear(const void* X, int64_t T, int64_t ldx, const w4a4_packed_weight* pw,
+                        void* workspace, size_t ws_bytes, void* Y, int64_t ldy, void* stream);
+
+/* The online layer from and to HOST memory: copies X_host (bf16 [T, d_in],
+ * dense rows; pinned memory gives an asynchronous copy) to X_dev, runs
+ * w4a4_linear, copies Y_dev back to Y_host (bf16 [T, d_out], dense rows), all
+ * on `stream`.  X_dev / Y_dev are caller-owned device buffers of those sizes.
+ * Returns once the work is enqueued; synchronise the stream before reading
+ * Y_host. */
+w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_weight* pw,
+                             void* X_dev, void* workspace, size_t ws_bytes, void* Y_dev,
+                             void* Y_host, void* stream);
+
+/* Synchronises `stream` and reports device-side failures recorded since the
+ * last clear: W4A4_OK, or W4A4_ERR_TIMEOUT if a bounded wait ran out (the
+ * affected output is incomplete).  *bits (may be NULL) receives the raw
+ * error word.  clear != 0 resets the word. */
+w4a4_status w4a4_last_error(void* stream, int clear, uint32_t* bits);
+
+/* Number of streaming multiprocessors of the current device (used to size
+ * persistent grids); 0 on error. */
+int w4a4_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A4_H */

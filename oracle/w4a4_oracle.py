@@ -276,7 +276,7 @@ def prep_activation(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray, J: np.ndarr
 # ----------------------------------------------------------------------------
 
 def pack_weight(W: np.ndarray, s: np.ndarray, O: np.ndarray, J: np.ndarray,
-                layout: int = LAYOUT_32x1):
+                layout: int = LAYOUT_32x1, row_chunk: int = 512):
     """Fold s into W, split off the O rows (columns here) in bf16, MXFP4-pack J.
 
     W: float32 values [d_out, d_in] (bf16-exact).  Returns a dict with
@@ -284,30 +284,36 @@ def pack_weight(W: np.ndarray, s: np.ndarray, O: np.ndarray, J: np.ndarray,
       sfb   uint8 [d_out, nblk]     E8M0 codes (32x32: the tile's code repeated
                                     on each of its 32 rows)
       w_hp  uint16 [d_out, k]       bfloat16 bits of the folded O columns
+    Rows are processed in chunks (a multiple of 32) only to bound memory.
     """
+    if layout not in (LAYOUT_32x1, LAYOUT_32x32):
+        raise ValueError("unknown layout")
     d_out = W.shape[0]
     kj = J.shape[0]
     nb = n_blocks(kj)
-    Wf = fold_weight(W.astype(np.float32), s.astype(np.float32)).astype(np.float32)
-    w_hp = f32_to_bf16_bits(Wf[:, O])
+    s = s.astype(np.float32)
     wq = np.zeros((d_out, nb * 16), np.uint8)
     sfb = np.zeros((d_out, nb), np.uint8)
-    if nb:
-        WJ = _pad_cols(Wf[:, J], nb * MX_BLOCK).reshape(d_out, nb, MX_BLOCK)
+    w_hp = np.zeros((d_out, O.shape[0]), np.uint16)
+    for r0 in range(0, d_out, row_chunk):
+        r1 = min(d_out, r0 + row_chunk)
+        Wf = fold_weight(W[r0:r1].astype(np.float32), s).astype(np.float32)   # fl32 products
+        w_hp[r0:r1] = f32_to_bf16_bits(Wf[:, O])
+        if not nb:
+            continue
+        WJ = _pad_cols(Wf[:, J], nb * MX_BLOCK).reshape(r1 - r0, nb, MX_BLOCK)
         if layout == LAYOUT_32x1:
             sc, codes = mxfp4_quantize_blocks(WJ)
-        elif layout == LAYOUT_32x32:
-            rows_pad = -(-d_out // 32) * 32
-            amax_rows = np.max(np.abs(WJ), axis=-1)                       # [d_out, nb]
-            amax_rows = np.concatenate(
-                [amax_rows, np.zeros((rows_pad - d_out, nb), np.float32)], axis=0)
-            tile_amax = amax_rows.reshape(rows_pad // 32, 32, nb).max(axis=1)  # [tiles, nb]
-            per_row = np.repeat(tile_amax, 32, axis=0)[:d_out]
-            sc, codes = mxfp4_quantize_blocks(WJ, per_row)
         else:
-            raise ValueError("unknown layout")
-        sfb[:] = sc
-        wq[:] = pack_nibbles(codes.reshape(d_out, nb * MX_BLOCK))
+            # one amax per 32 rows x 32 columns; rows past d_out count as zeros
+            amax_rows = np.max(np.abs(WJ), axis=-1)                          # [rows, nb]
+            pad = (-(r1 - r0)) % 32
+            amax_rows = np.concatenate([amax_rows, np.zeros((pad, nb), np.float32)], axis=0)
+            tile_amax = amax_rows.reshape(-1, 32, nb).max(axis=1)            # [tiles, nb]
+            per_row = np.repeat(tile_amax, 32, axis=0)[:r1 - r0]
+            sc, codes = mxfp4_quantize_blocks(WJ, per_row)
+        sfb[r0:r1] = sc
+        wq[r0:r1] = pack_nibbles(codes.reshape(r1 - r0, nb * MX_BLOCK))
     return {"wq": wq, "sfb": sfb, "w_hp": w_hp}
 
 
@@ -360,15 +366,16 @@ def linear_reference(X: np.ndarray, W: np.ndarray, alpha: float, k: int,
     return Y, {**c, **pw, **pa}
 
 
-def mma_sf_offset(r: int, kb: int, nblk: int) -> int:
+def mma_sf_offset(r, kb, nblk: int):
     """Byte offset of scale (row r, block kb) in the block-scaled MMA layout.
 
     The layout is the public one for Blackwell block-scaled MMAs (CUTLASS
     ``Sm1xxBlockScaledConfig``): 128-row x 4-block atoms of 512 bytes, atoms
     K-major, inside an atom row r sits at (r % 32) * 16 + ((r % 128) // 32) * 4
     and block kb at kb % 4.  ``nblk`` is the number of blocks per row of the
-    buffer (padded to a multiple of 4).  Used by tests to read GPU scale
-    buffers back into the canonical [rows, nblk] order.
+    buffer (padded to a multiple of 4).  Accepts integers or numpy integer
+    arrays.  Used by tests to read GPU scale buffers back into the canonical
+    [rows, nblk] order; it is a storage order, not part of the arithmetic.
     """
     atoms_k = -(-nblk // 4)
     return (((r // 128) * atoms_k + kb // 4) * 512 + (r % 32) * 16

@@ -1,0 +1,106 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every symbol include/w4a4.h declares, and validates arguments before any
+launch (invalid calls return an error status and enqueue nothing)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_mxfp4_outlier_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "w4a4.h")).read()
+    return sorted(set(re.findall(r"\b(w4a4_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(w4.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(w4.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings():
+    assert w4.abi_version() == 1
+    assert w4.status_string(w4.OK) == "ok"
+    assert "timed out" in w4.status_string(w4.ERR_TIMEOUT)
+
+
+def test_dims():
+    d = w4.get_dims(5120, 13824, 32)
+    assert (d.kj, d.kj_pad, d.nblk, d.k_pad, d.sfb_rows) == (5088, 5120, 160, 32, 13824)
+    d = w4.get_dims(13824, 5120, 64)
+    assert (d.kj, d.kj_pad, d.nblk, d.k_pad) == (13760, 13824, 432, 64)
+    d = w4.get_dims(512, 512, 8)
+    assert (d.kj_pad, d.k_pad, d.sfb_rows) == (512, 16, 512)
+    d = w4.get_dims(5120, 13824, 0)
+    assert (d.kj_pad, d.k_pad) == (5120, 0)
+    d = w4.get_dims(64, 48, 64)
+    assert (d.kj, d.kj_pad, d.nblk, d.sfb_rows) == (0, 0, 0, 256)
+
+
+def test_sizes():
+    b = w4.weight_sizes(5120, 13824, 32)
+    assert (b.wq, b.sfb, b.w_hp) == (13824 * 2560, 13824 * 160, 13824 * 32 * 2)
+    n = w4.workspace_size(4096, 5120, 13824, 32)
+    assert n == 4096 * 2560 + 4096 * 160 + 4096 * 32 * 2
+    assert w4.workspace_size(100, 512, 512, 8) >= 100 * 256 + 128 * 16 + 100 * 16 * 2
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 16, 0), w4.ERR_INVALID_ARG),
+    ((64, 16, 65), w4.ERR_INVALID_ARG),
+    ((60, 16, 0), w4.ERR_UNSUPPORTED_SHAPE),      # d_in % 8
+    ((64, 24, 0), w4.ERR_UNSUPPORTED_SHAPE),      # d_out % 16
+    ((70000, 16, 0), w4.ERR_UNSUPPORTED_SHAPE),   # d_in > 65535
+])
+def test_weight_sizes_rejects(args, status):
+    with pytest.raises(w4.W4A4Error) as e:
+        w4.weight_sizes(*args)
+    assert e.value.status == status
+
+
+def _raw_pw(d_in=64, d_out=32, k=4, layout=0, fake=0x1000):
+    return w4.PackedWeightC(d_in, d_out, k, layout, 0, fake, fake, fake, fake, fake, fake)
+
+
+def test_calls_validate_before_launch():
+    # Pointers here are never dereferenced: every call must fail validation.
+    pw = _raw_pw()
+    st = w4._prep_act(0x1000, 8, 63, ctypes.byref(pw), 0x1000, 0x1000, 0x1000, None)  # ldx < d_in
+    assert st == w4.ERR_INVALID_ARG
+    st = w4._prep_act(0x1000, 8, 68, ctypes.byref(pw), 0x1000, 0x1000, 0x1000, None)  # ldx % 8
+    assert st == w4.ERR_UNSUPPORTED_SHAPE
+    st = w4._prep_act(0x1001, 8, 64, ctypes.byref(pw), 0x1000, 0x1000, 0x1000, None)  # misaligned X
+    assert st == w4.ERR_UNSUPPORTED_SHAPE
+    st = w4._gemm_dual(0x1000, 0x1000, 0x1000, 8, ctypes.byref(pw), 0x1000, 31, None)  # ldy < d_out
+    assert st == w4.ERR_INVALID_ARG
+    st = w4._gemm_dual(0x1000, 0x1000, None, 8, ctypes.byref(pw), 0x1000, 32, None)  # xo missing, k>0
+    assert st == w4.ERR_INVALID_ARG
+    bad = _raw_pw(layout=7)
+    assert w4._gemm_dual(0x1000, 0x1000, 0x1000, 8, ctypes.byref(bad), 0x1000, 32, None) == w4.ERR_INVALID_ARG
+    st = w4._linear(0x1000, 8, 64, ctypes.byref(pw), 0x1000, 16, 0x1000, 32, None)  # workspace too small
+    assert st == w4.ERR_INVALID_ARG
+    assert w4._prep_act(0x1000, 8, 64, None, 0x1000, 0x1000, 0x1000, None) == w4.ERR_INVALID_ARG
+    # T == 0 is a valid no-op that launches nothing
+    assert w4._prep_act(None, 0, 64, ctypes.byref(pw), None, None, None, None) == w4.OK
+    assert w4._gemm_dual(None, None, None, 0, ctypes.byref(pw), None, 32, None) == w4.OK
+
+
+def test_calib_validation():
+    assert w4._calib_observe(0x1000, 4, 8, 4, 0x1000, 1, None) == w4.ERR_INVALID_ARG      # lda < cols
+    assert w4._calib_observe(0x1000, 4, 12, 12, 0x1000, 1, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._calib_observe(None, 4, 8, 8, 0x1000, 1, None) == w4.ERR_INVALID_ARG
+    f = 0x1000
+    assert w4._calib_finalize(f, f, 64, 0.0, 4, f, f, f, f, f, None) == w4.ERR_INVALID_ARG   # alpha
+    assert w4._calib_finalize(f, f, 64, 1.0, 4, f, f, f, f, f, None) == w4.ERR_INVALID_ARG
+    assert w4._calib_finalize(f, f, 64, 0.5, 65, f, f, f, f, f, None) == w4.ERR_INVALID_ARG  # k > d_in
+    assert w4._calib_finalize(f, f, 64, 0.5, 4, f, f, f, None, f, None) == w4.ERR_INVALID_ARG  # O missing
+    assert w4._calib_finalize(f, f, 20000, 0.5, 4, f, f, f, f, f, None) == w4.ERR_UNSUPPORTED_SHAPE

@@ -1,0 +1,77 @@
+"""Host-side pieces of bench.py on CPU: the multi-rank plumbing over gloo with
+world size 2 (barrier, max over ranks, whole-job aggregation) and the
+reference arm (the CPU oracle), which only rank 0 runs and prints."""
+import io
+import json
+import multiprocessing as mp
+import os
+import socket
+
+from contextlib import redirect_stdout
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    import torch
+    import torch.distributed as dist
+    w, r, _ = bench.dist_env()
+    active = bench.dist_init("gloo", w, r, timeout_s=60)
+    bench.dist_barrier(active)
+    step_s = 0.5 + rank            # rank 1 is the slow one
+    m = bench.dist_max(step_s, active, torch.device("cpu"))
+    q.put((rank, active, m, bench.aggregate(100.0, w, m)))
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_and_aggregate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[0] for r in res] == [0, 1]
+    for rank, active, m, agg in res:
+        assert active and m == 1.5                      # max over ranks
+        assert agg == 100.0 * 2 / 1.5                   # all ranks' units / slowest time
+
+
+def test_single_rank_is_not_distributed():
+    assert bench.dist_init("gloo", 1, 0) is False
+    assert bench.dist_max(3.0, False, None) == 3.0
+
+
+def test_reference_arm_prints_on_rank0_only(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
+    assert buf.getvalue() == ""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+
+
+

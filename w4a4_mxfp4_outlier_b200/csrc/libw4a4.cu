@@ -1,0 +1,8 @@
+// Single translation unit of libw4a4: every kernel and the C-ABI are
+// compiled together so device globals (the error word) are shared without
+// relocatable device code.
+#include "w4a4_api.cu"
+#include "calib.cu"
+#include "pack.cu"
+#include "prep.cu"
+#include "gemm.cu"

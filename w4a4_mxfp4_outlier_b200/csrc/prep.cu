@@ -1,0 +1,230 @@
+// Online activation preparation: one pass over X that divides by s (as a
+// multiply by inv_s), gathers the outlier columns into a dense bf16 matrix
+// and MXFP4-encodes the compacted remaining columns, writing E2M1 codes and
+// E8M0 scales directly in the layout the block-scaled tensor-core MMA reads.
+//
+// Method: paper review "W4A4 Quantization for Inference on Wan2.2-I2V-A14B",
+// sec. 3.2 ("at inference activations are first divided by s, then
+// quantised") and sec. 3.3 (X_J in 4 bits, X_O in high precision).
+//
+// Design (HBM-bound; 2 bytes read and ~0.56 bytes written per element):
+//  * persistent grid, one CTA per SM; CTA b handles rows b, b+G, b+2G, ...
+//  * warp 0 lane 0 streams whole rows into a ring of shared-memory buffers
+//    with cp.async.bulk (completion counted on an mbarrier per buffer);
+//  * each consumer thread owns CH chunks of 8 consecutive compacted columns
+//    for the whole kernel: their source column and inv_s live in registers;
+//  * four lanes form one 32-element MX block (amax by two xor shuffles);
+//    a warp covers 256 columns and stores 128 contiguous code bytes;
+//  * the 8 elements of a chunk are gathered pair by pair in an order rotated
+//    by (lane / 8) % 4 so the 32 lanes of a warp hit 32 different banks;
+//  * the padding columns (p >= kj) and padding outlier slots read a zero
+//    slot stored after each row buffer, so they encode as +0 with no branch.
+#include "w4a4_internal.h"
+
+namespace w4a4 {
+
+constexpr int kPrepMaxThreads = 1024;
+
+template <int CH>
+__global__ void __launch_bounds__(kPrepMaxThreads, 1)
+    prep_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t ldx, int d_in,
+                const float* __restrict__ inv_s, const int32_t* __restrict__ O,
+                const int32_t* __restrict__ jmap, int k, int k_pad, int kj, int nchunks, int nblk,
+                uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa, uint32_t* __restrict__ xo,
+                int stages, int stage_bytes) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
+  uint64_t* empty = full + stages;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + stages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NT = blockDim.x - 32;           // consumer threads (multiple of 32)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NT / 32);
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  for (int s = threadIdx.x; s < stages; s += blockDim.x)
+    *reinterpret_cast<uint4*>(smem + static_cast<size_t>(s) * stage_bytes + 2 * d_in) =
+        make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+
+  const int64_t nrows = T > blockIdx.x ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
+      int64_t issued = 0;
+      for (int64_t i = 0; i < nrows; ++i) {
+        const int s = static_cast<int>(i % stages);
+        const uint32_t ph = static_cast<uint32_t>((i / stages) & 1);
+        if (i >= stages && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
+          break;
+        const int64_t r = blockIdx.x + i * gridDim.x;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_load(smem + static_cast<size_t>(s) * stage_bytes, X + r * ldx, bytes, &full[s]);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // do not leave bulk copies in flight into shared memory we give back
+        const int64_t first = issued > stages ? issued - stages : 0;
+        for (int64_t i = first; i < issued; ++i)
+          mbar_wait_bounded(&full[i % stages], static_cast<uint32_t>((i / stages) & 1), nullptr,
+                            DEVERR_TIMEOUT_PREP);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int ct = threadIdx.x - 32;
+  const int rot = (lane >> 3) & 3;
+  uint32_t idx[CH][4];     // two 16-bit source columns per register (pair order rotated)
+  float isv[CH][8];
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int chunk = ct + c * NT;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int qq = (q + rot) & 3;
+      const int p0 = chunk * 8 + 2 * qq;
+      uint32_t src0 = static_cast<uint32_t>(d_in), src1 = static_cast<uint32_t>(d_in);
+      float i0 = 1.f, i1 = 1.f;
+      if (chunk < nchunks && p0 < kj) {
+        src0 = static_cast<uint32_t>(jmap[p0]);
+        i0 = inv_s[src0];
+      }
+      if (chunk < nchunks && p0 + 1 < kj) {
+        src1 = static_cast<uint32_t>(jmap[p0 + 1]);
+        i1 = inv_s[src1];
+      }
+      idx[c][q] = src0 | (src1 << 16);
+      isv[c][2 * q] = i0;
+      isv[c][2 * q + 1] = i1;
+    }
+  }
+  const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
+  const int xo_row = k_pad >> 1;                            // bf16 pairs per row of X_O
+
+  for (int64_t i = 0; i < nrows; ++i) {
+    const int s = static_cast<int>(i % stages);
+    const uint32_t ph = static_cast<uint32_t>((i / stages) & 1);
+    if (!mbar_wait_bounded(&full[s], ph, abort_flag, DEVERR_TIMEOUT_PREP)) break;
+    const int64_t r = blockIdx.x + i * gridDim.x;
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(s) * stage_bytes);
+
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int chunk = ct + c * NT;
+      if (chunk < nchunks) {                // uniform per warp (nchunks % 32 == 0)
+        float v[8];
+        float amax = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t pr = idx[c][q];
+          const float x0 = __uint_as_float(static_cast<uint32_t>(row[pr & 0xFFFFu]) << 16);
+          const float x1 = __uint_as_float(static_cast<uint32_t>(row[pr >> 16]) << 16);
+          v[2 * q] = __fmul_rn(x0, isv[c][2 * q]);
+          v[2 * q + 1] = __fmul_rn(x1, isv[c][2 * q + 1]);
+          amax = fmaxf(amax, fmaxf(fabsf(v[2 * q]), fabsf(v[2 * q + 1])));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        const uint32_t code = mx_scale_code(amax);
+        const float inv = mx_inv_scale(code);
+        uint32_t w = cvt_e2m1x8(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv, v[4] * inv,
+                                v[5] * inv, v[6] * inv, v[7] * inv);
+        w = __funnelshift_l(w, w, 8 * rot);   // undo the pair rotation
+        *reinterpret_cast<uint32_t*>(aq + r * aq_row + 4 * static_cast<int64_t>(chunk)) = w;
+        const uint32_t c4 = __shfl_down_sync(0xFFFFFFFFu, code, 4);
+        const uint32_t c8 = __shfl_down_sync(0xFFFFFFFFu, code, 8);
+        const uint32_t c12 = __shfl_down_sync(0xFFFFFFFFu, code, 12);
+        if ((lane & 15) == 0) {
+          const int64_t kb = chunk >> 2;       // multiple of 4
+          *reinterpret_cast<uint32_t*>(sfa + sf_offset(r, kb, nblk)) =
+              code | (c4 << 8) | (c8 << 16) | (c12 << 24);
+        }
+      }
+    }
+    for (int i2 = ct; i2 < xo_row; i2 += NT) {
+      const int o0 = 2 * i2;
+      const int src0 = o0 < k ? O[o0] : d_in;
+      const int src1 = o0 + 1 < k ? O[o0 + 1] : d_in;
+      const float s0 = o0 < k ? inv_s[src0] : 1.f;
+      const float s1 = o0 + 1 < k ? inv_s[src1] : 1.f;
+      const float v0 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src0]) << 16), s0);
+      const float v1 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src1]) << 16), s1);
+      const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(v0));
+      const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(v1));
+      xo[r * xo_row + i2] = b0 | (b1 << 16);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
+struct PrepPlan {
+  int ch, nt, stages, stage_bytes;
+  size_t smem;
+};
+
+static PrepPlan plan_prep(const Geometry& g) {
+  PrepPlan p{};
+  const int nchunks = static_cast<int>(g.kj_pad / 8);
+  const int max_nt = kPrepMaxThreads - 32;
+  p.ch = 1;
+  while (p.ch < 4 && (nchunks + p.ch - 1) / p.ch > max_nt) p.ch *= 2;
+  int nt = (nchunks + p.ch - 1) / p.ch;
+  nt = static_cast<int>(round_up(nt < 32 ? 32 : nt, 32));
+  p.nt = nt;
+  p.stage_bytes = static_cast<int>(round_up(2 * g.d_in + 16, 128));
+  int st = (160 * 1024) / p.stage_bytes;
+  p.stages = st < 2 ? 2 : (st > 8 ? 8 : st);
+  p.smem = static_cast<size_t>(p.stages) * p.stage_bytes + 2 * p.stages * 8 + 16;
+  return p;
+}
+
+bool prep_supported(const Geometry& g) {
+  if (g.d_in > 65535) return false;
+  const int nchunks = static_cast<int>(g.kj_pad / 8);
+  if (nchunks > 4 * (kPrepMaxThreads - 32)) return false;
+  return plan_prep(g).smem <= 227 * 1024;
+}
+
+template <int CH>
+static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, int64_t T,
+                                  int64_t ldx, const float* inv_s, const int32_t* O,
+                                  const int32_t* jmap, const Geometry& g, uint8_t* aq,
+                                  uint8_t* sfa, void* xo, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(prep_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(p.smem));
+  if (e != cudaSuccess) return e;
+  prep_kernel<CH><<<grid, p.nt + 32, p.smem, stream>>>(
+      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
+      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
+      static_cast<int>(g.kj_pad / 8), static_cast<int>(g.nblk), aq, sfa,
+      static_cast<uint32_t*>(xo), p.stages, p.stage_bytes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
+                        const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
+                        uint8_t* sfa, void* xo, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const PrepPlan p = plan_prep(g);
+  const int sms = device_num_sms();
+  const int grid = static_cast<int>(T < sms ? T : sms);
+  switch (p.ch) {
+    case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+    case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+  }
+}
+
+}  // namespace w4a4

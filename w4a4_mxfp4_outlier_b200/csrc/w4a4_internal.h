@@ -1,0 +1,63 @@
+// Internal declarations shared by the translation units of libw4a4.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "w4a4_device.cuh"
+
+namespace w4a4 {
+
+constexpr int kKTileElems = 256;   // compacted 4-bit K elements per GEMM K tile (128 bytes)
+constexpr int kSfbRowPad = 256;    // scale rows of B are padded to the GEMM N tile
+constexpr int kSfaRowPad = 128;    // scale rows of A are padded to the GEMM M tile
+
+struct Geometry {
+  int64_t d_in, d_out, k;
+  int64_t kj, kj_pad, nblk, k_pad, sfb_rows;
+};
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+inline Geometry make_geometry(int64_t d_in, int64_t d_out, int64_t k) {
+  Geometry g;
+  g.d_in = d_in;
+  g.d_out = d_out;
+  g.k = k;
+  g.kj = d_in - k;
+  g.kj_pad = round_up(g.kj, kKTileElems);
+  g.nblk = g.kj_pad / 32;
+  g.k_pad = round_up(k, 16);
+  g.sfb_rows = round_up(d_out, kSfbRowPad);
+  return g;
+}
+
+// Byte offset of the scale of (row r, block b) in the block-scaled MMA
+// layout with nblk blocks per row (nblk a multiple of 4): 512-byte atoms of
+// 128 rows x 4 blocks, K-major; inside an atom (r%32)*16 + ((r%128)/32)*4 + b%4.
+__host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t b, int64_t nblk) {
+  return (((r >> 7) * (nblk >> 2) + (b >> 2)) << 9) + ((r & 31) << 4) + (((r & 127) >> 5) << 2) +
+         (b & 3);
+}
+
+int device_num_sms();
+
+cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
+                             int reset, cudaStream_t stream);
+cudaError_t launch_finalize(const float* act, const float* wsc, int d_in, double alpha, int k,
+                            float* s, float* inv_s, float* score, int32_t* O, int32_t* jmap,
+                            cudaStream_t stream);
+int finalize_max_d();
+cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,
+                        const int32_t* jmap, const Geometry& g, int layout, uint8_t* wq,
+                        uint8_t* sfb, void* w_hp, cudaStream_t stream);
+cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
+                        const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
+                        uint8_t* sfa, void* xo, cudaStream_t stream);
+bool prep_supported(const Geometry& g);
+cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                        const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
+                        void* Y, int64_t ldy, cudaStream_t stream);
+
+}  // namespace w4a4

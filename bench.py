@@ -287,7 +287,7 @@ def run_gpu(args):
     e2e = run_e2e(args, runs, w4, device, active) if not args.no_e2e else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(layers, runs)
+        cpu = cpu_baseline(layers, runs, rows=256, outs=1024)
 
     if rank == 0:
         out = {
@@ -461,7 +461,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="full", choices=["full", "ffn0", "ffn2", "tiny", "sweep"])
+    ap.add_argument("--workload", default="full",
+                    choices=["full", "full_up", "full_down", "mid_up", "ffn0", "ffn2", "tiny", "sweep"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

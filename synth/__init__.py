@@ -115,11 +115,16 @@ def sweep_layers():
     return out
 
 
+MID_UP = Layer("mid_up_T16384", 16384, 5120, 13824, 0.6, 32, 0, X_UP, W_UP)
+
 WORKLOADS = {
     "tiny": [TINY],
     "ffn0": [FFN0],
     "ffn2": [FFN2],
     "full": [FULL_UP, FULL_DOWN],
+    "full_up": [FULL_UP],
+    "full_down": [FULL_DOWN],
+    "mid_up": [MID_UP],
     "sweep": sweep_layers(),
 }
 

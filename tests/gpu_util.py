@@ -17,11 +17,12 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def sf_canonical(flat: torch.Tensor, rows: int, nblk_lib: int, nblk_ref: int) -> np.ndarray:
-    """Scale bytes in the MMA layout -> [rows, nblk_ref] canonical order, plus
-    the padding blocks [rows, nblk_ref:nblk_lib] for a zero check."""
+def sf_canonical(flat: torch.Tensor, rows, nblk_lib: int, nblk_ref: int) -> np.ndarray:
+    """Scale bytes in the MMA layout -> canonical [rows, nblk_lib] order (the
+    blocks past nblk_ref are padding, returned for a zero check).  ``rows`` is
+    a row count or an array of row indices."""
     buf = flat.cpu().numpy()
-    r = np.arange(rows)[:, None]
+    r = (np.arange(rows) if np.isscalar(rows) else np.asarray(rows))[:, None]
     kb = np.arange(nblk_lib)[None, :]
     return buf[orc.mma_sf_offset(r, kb, nblk_lib)]
 

@@ -1,0 +1,54 @@
+"""Parity at the full 720x1280x61 token count (T = 57600), in the launch
+configuration bench.py times (calib_observe, calib_finalize, pack_weight,
+prep_act, gemm_dual on the whole tensors), checked on what the oracle can
+afford: the calibration scales over all of X (in row chunks), the packed
+weight in full, and the activation codes and Y on 1024 seeded sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import w4a4_mxfp4_outlier_b200 as w4
+from oracle import w4a4_oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("L", [synth.FULL_UP, synth.FULL_DOWN], ids=lambda L: L.name)
+def test_full_size_sampled(L):
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
+    act = w4.alloc_act(L.T, pw)
+    Y = torch.empty((L.T, L.d_out), dtype=torch.bfloat16, device="cuda")
+    w4.prep_act(X, pw, act)
+    w4.gemm_dual(act, L.T, pw, Y)
+    st, bits = w4.last_error()
+    assert st == w4.OK, f"device error word {bits:#x}"
+
+    # calibration over every token, chunked on the host
+    run = None
+    for r0 in range(0, L.T, 4096):
+        run = orc.col_absmax(gu.to_np_f32(X[r0:r0 + 4096]), run)
+    np.testing.assert_array_equal(pw.act_scale.cpu().numpy(), run)
+    Wn = gu.to_np_f32(W)
+    np.testing.assert_array_equal(pw.w_scale.cpu().numpy(), orc.col_absmax(Wn))
+    c = gu.oracle_calib_from_gpu(pw)
+    np.testing.assert_array_equal(pw.O.cpu().numpy(), c["O"])
+
+    ref_w = orc.pack_weight(Wn, c["s"], c["O"], c["J"], L.layout)
+    d = pw.dims
+    nb = ref_w["sfb"].shape[1]
+    np.testing.assert_array_equal(pw.wq.view(L.d_out, -1).cpu().numpy()[:, :nb * 16], ref_w["wq"])
+
+    rows = synth.sample_rows(L.T, 1024).numpy()
+    ridx = torch.from_numpy(rows).cuda()
+    ref_a = orc.prep_activation(gu.to_np_f32(X[ridx]), c["inv_s"], c["O"], c["J"])
+    np.testing.assert_array_equal(act.aq[ridx].cpu().numpy()[:, :nb * 16], ref_a["aq"])
+    sfa = gu.sf_canonical(act.sfa, rows, d.nblk, nb)
+    np.testing.assert_array_equal(sfa[:, :nb], ref_a["sfa"])
+    np.testing.assert_array_equal(gu.bf16_bits(act.xo[ridx])[:, :L.k], ref_a["xo"])
+
+    Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
+                                    ref_w["sfb"], ref_w["w_hp"])
+    gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, L.name)

@@ -3,7 +3,7 @@
 // allocates device memory.
 #include <cstring>
 
-#include "../../include/w4a4.h"
+#include "w4a4.h"
 #include "w4a4_internal.h"
 
 namespace w4a4 {
@@ -135,6 +135,7 @@ w4a4_status w4a4_pack_weight(const void* W, int64_t ldw, const float* s,
   w4a4_status st = check_pw(pw, &g);
   if (st != W4A4_OK) return st;
   if (W == nullptr || s == nullptr || ldw < g.d_in) return W4A4_ERR_INVALID_ARG;
+  if (ldw % 8 != 0 || !aligned16(W)) return W4A4_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(launch_pack(W, ldw, s, pw->O, pw->jmap, g, pw->layout, pw->wq, pw->sfb,
                                pw->w_hp, static_cast<cudaStream_t>(stream)));
 }

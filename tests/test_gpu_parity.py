@@ -32,7 +32,9 @@ MID = synth.Layer("mid_k256_32x32", 640, 5120, 1024, 0.7, 256, 1, synth.X_UP, sy
 FFN0 = synth.FFN0
 FFN2 = synth.FFN2
 
-SMALL = [TINY, RAGGED, RAGGED32, K0, KFULL, T1]
+SINGLE = RAGGED.with_(name="ragged_T100_single_cta", T=100, k=5)   # T <= 128: single-CTA GEMM
+
+SMALL = [TINY, RAGGED, RAGGED32, K0, KFULL, T1, SINGLE]
 
 
 def _calibrate(L):

@@ -22,9 +22,10 @@
 //   warps 2-9   epilogue: each warp drains 32 lanes x 128 columns of the
 //               accumulator (tcgen05.ld), releases it, converts to bf16 and
 //               stores its rows of Y.
-// Scale factors sit in tensor memory columns 256..279, rewritten for each
-// K tile; tcgen05.cp and tcgen05.mma issued by one thread execute in order,
-// so a rewrite never overtakes the MMAs that read the previous scales.
+// Scale factors sit in tensor memory columns 256..279 and 288..311, the two
+// buffers alternating by K tile, so the copy of one tile's scales does not
+// have to wait for the MMAs still reading the previous tile's (tcgen05.cp
+// and tcgen05.mma issued by one thread execute in order in any case).
 // Every wait is bounded (about 2 s); a role that gives up sets the device
 // error word and an abort flag the others poll, and all roles then exit
 // through the same teardown (drain in-flight copies / MMAs, free tensor
@@ -49,6 +50,7 @@ constexpr int GEMM_THREADS = 32 * (2 + NUM_EPI_WARPS);
 constexpr int TMEM_COLS = 512;
 constexpr int TMEM_SFA_COL = 256;             // 2 atoms x 4 columns
 constexpr int TMEM_SFB_COL = 264;             // 2 atoms x 8 columns
+constexpr int TMEM_SF_BUF = 32;               // scale buffers alternate by K tile: +0 / +32 columns
 constexpr int GROUP_M = 16;                   // tile raster: 16 M tiles per sweep of N
 
 struct GemmSmem {
@@ -130,22 +132,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (warp == 0) {
     // ============================ TMA producer ============================
-    if (lane == 0) {
-      uint32_t it = 0;                 // global K-tile counter (ring position)
-      uint32_t issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        int tm, tn;
-        tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
-        const int m0 = tm * BM, n0 = tn * BN;
-        for (int kt = 0; kt < nkt; ++kt, ++it) {
-          const int s = static_cast<int>(it % STAGES);
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (it >= STAGES &&
-              !mbar_wait_bounded(&sm.empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
-            ok = false;
-            break;
-          }
+    // The whole warp runs the loop and waits; one elected lane issues.
+    uint32_t it = 0;                   // global K-tile counter (ring position)
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      int tm, tn;
+      tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
+      const int m0 = tm * BM, n0 = tn * BN;
+      for (int kt = 0; kt < nkt; ++kt, ++it) {
+        const int s = static_cast<int>(it % STAGES);
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (it >= STAGES &&
+            !warp_wait_bounded(&sm.empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           uint8_t* st = sm.stage[s];
           if (kt < args.kt_o) {
             mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
@@ -165,39 +168,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + rb * 1024, sb, 1024, &sm.full[s]);
             }
           }
-          issued = it + 1;
         }
-      }
-      if (*abort_flag) {
-        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
-        for (uint32_t i = first; i < issued; ++i)
-          mbar_wait_bounded(&sm.full[i % STAGES], (i / STAGES) & 1u, nullptr,
-                            DEVERR_TIMEOUT_PRODUCER);
+        __syncwarp();
+        issued = it + 1;
       }
     }
+    if (lane == 0 && *abort_flag) {
+      // wait for the copies still in flight, so none lands after teardown
+      const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+      for (uint32_t i = first; i < issued; ++i)
+        mbar_wait_bounded(&sm.full[i % STAGES], (i / STAGES) & 1u, nullptr, DEVERR_TIMEOUT_PRODUCER);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ============================ MMA issuer ==============================
-    if (lane == 0) {
-      const uint32_t idesc_o = idesc_bf16(BM, BN);
-      const uint32_t tsfa = tmem + TMEM_SFA_COL;
-      const uint32_t tsfb = tmem + TMEM_SFB_COL;
-      uint32_t it = 0, tcount = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-        // wait until the epilogue has drained the accumulator of the previous tile
-        if (!mbar_wait_bounded(&sm.acc_empty, (tcount & 1u) ^ 1u, abort_flag, DEVERR_TIMEOUT_MMA)) {
+    // The whole warp runs the loop and waits; one elected lane issues.
+    const uint32_t idesc_o = idesc_bf16(BM, BN);
+    const uint32_t tsfa = tmem + TMEM_SFA_COL;
+    const uint32_t tsfb = tmem + TMEM_SFB_COL;
+    uint32_t it = 0, tcount = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+      // wait until the epilogue has drained the accumulator of the previous tile
+      if (!warp_wait_bounded(&sm.acc_empty, (tcount & 1u) ^ 1u, abort_flag, DEVERR_TIMEOUT_MMA)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int kt = 0; kt < nkt; ++kt, ++it) {
+        const int s = static_cast<int>(it % STAGES);
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!warp_wait_bounded(&sm.full[s], ph, abort_flag, DEVERR_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int kt = 0; kt < nkt; ++kt, ++it) {
-          const int s = static_cast<int>(it % STAGES);
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&sm.full[s], ph, abort_flag, DEVERR_TIMEOUT_MMA)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        if (elect_one()) {
           const uint32_t a_addr = smem_u32(sm.stage[s]);
           const uint32_t b_addr = a_addr + A_BYTES;
           if (kt < args.kt_o) {
@@ -207,33 +213,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               mma_bf16(tmem, sdesc_kmajor_sw128(a_addr + kk * 32), sdesc_kmajor_sw128(b_addr + kk * 32),
                        idesc_o, (kt | kk) != 0 ? 1u : 0u);
           } else {
+            // scales of this K tile go to the buffer the previous tile's MMAs
+            // do not read, so the copy need not wait for them
+            const uint32_t buf = static_cast<uint32_t>(it & 1u) * TMEM_SF_BUF;
+            const uint32_t sa = tsfa + buf, sb = tsfb + buf;
             const uint32_t sfa_s = b_addr + B_BYTES;
             const uint32_t sfb_s = sfa_s + SFA_BYTES;
-            tc_cp_32x128b_warpx4(tsfa + 0, sdesc_sf_rows16(sfa_s));
-            tc_cp_32x128b_warpx4(tsfa + 4, sdesc_sf_rows16(sfa_s + 512));
-            tc_cp_32x128b_warpx4(tsfb + 0, sdesc_sf_rows16(sfb_s));
-            tc_cp_32x128b_warpx4(tsfb + 8, sdesc_sf_rows16(sfb_s + 512));
-            tc_cp_32x128b_warpx4(tsfb + 4, sdesc_sf_rows16(sfb_s + 1024));
-            tc_cp_32x128b_warpx4(tsfb + 12, sdesc_sf_rows16(sfb_s + 1536));
+            tc_cp_32x128b_warpx4(sa + 0, sdesc_sf_rows16(sfa_s));
+            tc_cp_32x128b_warpx4(sa + 4, sdesc_sf_rows16(sfa_s + 512));
+            tc_cp_32x128b_warpx4(sb + 0, sdesc_sf_rows16(sfb_s));
+            tc_cp_32x128b_warpx4(sb + 8, sdesc_sf_rows16(sfb_s + 512));
+            tc_cp_32x128b_warpx4(sb + 4, sdesc_sf_rows16(sfb_s + 1024));
+            tc_cp_32x128b_warpx4(sb + 12, sdesc_sf_rows16(sfb_s + 1536));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t atom = static_cast<uint32_t>(kk >> 1);
               const uint32_t id = static_cast<uint32_t>((kk & 1) * 2);
               mma_mxf4(tmem, sdesc_kmajor_sw128(a_addr + kk * 32),
                        sdesc_kmajor_sw128(b_addr + kk * 32), idesc_mxf4(BM, BN, id, id),
-                       (tsfa + 4 * atom) | (id << 30), (tsfb + 8 * atom) | (id << 30),
+                       (sa + 4 * atom) | (id << 30), (sb + 8 * atom) | (id << 30),
                        (kt | kk) != 0 ? 1u : 0u);
             }
           }
           tc_commit(&sm.empty[s]);     // stage is free once these MMAs have read it
         }
-        if (!ok) break;
-        tc_commit(&sm.acc_full);       // accumulator complete
+        __syncwarp();
       }
-      // wait for every MMA / copy this thread issued before tensor memory is freed
-      tc_commit(&sm.drain);
-      mbar_wait_bounded(&sm.drain, 0u, nullptr, DEVERR_TIMEOUT_MMA);
+      if (!ok) break;
+      if (elect_one()) tc_commit(&sm.acc_full);   // accumulator complete
+      __syncwarp();
     }
+    // wait for every MMA / copy issued before tensor memory is freed (the
+    // elected lane is the same one that issued them)
+    if (elect_one()) tc_commit(&sm.drain);
+    __syncwarp();
+    mbar_wait_bounded(&sm.drain, 0u, nullptr, DEVERR_TIMEOUT_MMA);
+    __syncwarp();
   } else {
     // ============================ epilogue ================================
     const int ew = warp - 2;                 // 0..7
@@ -294,6 +309,309 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
 }
 
+// ===========================================================================
+// CTA-pair kernel (tcgen05 cta_group::2): a cluster of two CTAs computes a
+// 256 x 256 output tile.  CTA r of the pair stages its own 128 token rows of
+// A and its own 128 output rows of B (so B's shared-memory traffic per SM
+// halves against the single-CTA kernel), plus its A scales and all 256 rows of
+// B scales; the leader CTA (rank 0) issues the M=256 MMAs for both.  Each
+// CTA's tensor memory holds the accumulator of its 128 rows and, in the same
+// layout as the single-CTA kernel, its scale factors.
+//
+// Synchronisation: the TMA copies of both CTAs complete on the leader's
+// "full" barrier (the leader posts the expected byte count of both); the
+// leader's MMA completions are multicast to the "empty" and "acc_full"
+// barriers of both CTAs; the epilogue warps of both CTAs arrive on the
+// leader's "acc_empty".  No load uses cluster multicast.
+// ===========================================================================
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = 128 * KT_BYTES;     // own 128 token rows
+constexpr int P_B_BYTES = 128 * KT_BYTES;     // own 128 output rows
+constexpr int P_SFA_BYTES = 1024;             // own 128 rows x 8 blocks
+constexpr int P_SFB_BYTES = 2048;             // all 256 output rows x 8 blocks
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;
+constexpr int P_EPI_ARRIVALS = 2 * NUM_EPI_WARPS;
+
+struct PairSmem {
+  uint8_t stage[P_STAGES][P_STAGE_BYTES];
+  uint64_t full[P_STAGES];     // leader's counts the bytes of both CTAs
+  uint64_t empty[P_STAGES];    // both CTAs: MMA commit, multicast
+  uint64_t acc_full;           // both CTAs: MMA commit, multicast
+  uint64_t acc_empty;          // leader: epilogue warps of both CTAs
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_dual_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
+                          const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                          const GemmArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PairSmem& sm = *reinterpret_cast<PairSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  volatile uint32_t* abort_flag = &sm.abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();          // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int ntiles = args.tiles_m * args.tiles_n;   // 256 x 256 tiles
+  const int nkt = args.kt_o + args.kt_j;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, P_EPI_ARRIVALS);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0u;
+    fence_barrier_init();
+    if (args.kt_j > 0) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+      prefetch_tmap(&tm_sfa);
+      prefetch_tmap(&tm_sfb);
+    }
+    if (args.kt_o > 0) {
+      prefetch_tmap(&tm_ao);
+      prefetch_tmap(&tm_bo);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();          // barriers of both CTAs are initialised
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ============================ TMA producer (both CTAs) ================
+    // The whole warp runs the loop and waits; one elected lane issues.
+    uint32_t issued = 0;
+    bool ok = true;
+    const int atoms_k = args.nblk >> 2;
+    uint32_t it = 0, s = 0, ph = 0;
+    for (int t = pair; t < ntiles && ok; t += npairs) {
+      int tm, tn;
+      tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
+      const int m_rows = tm * 256 + 128 * static_cast<int>(rank);
+      const int n_rows = tn * 256 + 128 * static_cast<int>(rank);
+      for (int kt = 0; kt < nkt; ++kt, ++it) {
+        if (it >= P_STAGES &&
+            !warp_wait_bounded(&sm.empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          uint8_t* st = sm.stage[s];
+          const uint32_t full_leader = mapa_shared(smem_u32(&sm.full[s]), 0);
+          if (kt < args.kt_o) {
+            // the leader's barrier expects the bytes of both CTAs
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_BYTES + P_B_BYTES));
+            tma_load_2d_pair(st, &tm_ao, full_leader, kt * 64, m_rows);
+            tma_load_2d_pair(st + P_A_BYTES, &tm_bo, full_leader, kt * 64, n_rows);
+          } else {
+            const int kj = kt - args.kt_o;
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * P_STAGE_BYTES);
+            tma_load_2d_pair(st, &tm_a, full_leader, kj * KT_BYTES, m_rows);
+            tma_load_2d_pair(st + P_A_BYTES, &tm_b, full_leader, kj * KT_BYTES, n_rows);
+            // scale atoms: 256-byte rows of the scale buffers, 4 rows (1 KB) per copy
+            const int ya = ((2 * tm + static_cast<int>(rank)) * atoms_k + 2 * kj) * 2;
+            tma_load_2d_pair(st + P_A_BYTES + P_B_BYTES, &tm_sfa, full_leader, 0, ya);
+            for (int rb = 0; rb < 2; ++rb) {
+              const int yb = ((2 * tn + rb) * atoms_k + 2 * kj) * 2;
+              tma_load_2d_pair(st + P_A_BYTES + P_B_BYTES + P_SFA_BYTES + rb * 1024, &tm_sfb,
+                               full_leader, 0, yb);
+            }
+          }
+        }
+        __syncwarp();
+        issued = it + 1;
+        if (++s == P_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      if (rank == 0) {
+        // wait for the stages posted in the last ring's worth of K tiles, so
+        // no copy lands after teardown (earlier ones were consumed)
+        const uint32_t first = issued > P_STAGES ? issued - P_STAGES : 0;
+        for (uint32_t i = first; i < issued; ++i)
+          mbar_wait_bounded(&sm.full[i % P_STAGES], (i / P_STAGES) & 1u, nullptr,
+                            DEVERR_TIMEOUT_PRODUCER);
+      }
+      spin_ns(50000);            // the peer CTA's copies land on the leader's barriers
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================ MMA issuer (leader) =====================
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // tcgen05 instructions.  The issue path is latency-critical, so the loop
+    // only adds precomputed deltas: descriptors of stage 0 advanced by
+    // STAGE_DESC per stage, K offsets folded into unrolled constants,
+    // counters instead of divisions.
+    if (rank == 0) {
+      constexpr uint64_t STAGE_DESC = P_STAGE_BYTES >> 4;    // descriptor step per stage
+      const uint32_t st0 = smem_u32(sm.stage[0]);
+      const uint64_t da0 = sdesc_kmajor_sw128(st0);
+      const uint64_t db0 = sdesc_kmajor_sw128(st0 + P_A_BYTES);
+      const uint64_t dsa0 = sdesc_sf_rows16(st0 + P_A_BYTES + P_B_BYTES);
+      const uint64_t dsb0 = sdesc_sf_rows16(st0 + P_A_BYTES + P_B_BYTES + P_SFA_BYTES);
+      constexpr uint32_t ID_O = idesc_bf16(256, 256);
+      constexpr uint32_t ID_J0 = idesc_mxf4(256, 256, 0, 0);
+      constexpr uint32_t ID_J2 = idesc_mxf4(256, 256, 2, 2);
+      const uint32_t tsfa = tmem + TMEM_SFA_COL;
+      const uint32_t tsfb = tmem + TMEM_SFB_COL;
+      const int kt_o = args.kt_o, kt_j = args.kt_j;
+      const int nk_last_o = (args.k_pad - (kt_o - 1) * 64) / 16;   // K=16 steps in the last bf16 tile
+      uint32_t s = 0, ph = 0, buf = 0, tcount = 0;
+      uint64_t soff = 0;                 // STAGE_DESC * s
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs, ++tcount) {
+        if (!warp_wait_bounded(&sm.acc_empty, (tcount & 1u) ^ 1u, abort_flag, DEVERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t acc = 0;
+        for (int kt = 0; kt < kt_o; ++kt) {
+          if (!warp_wait_bounded(&sm.full[s], ph, abort_flag, DEVERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const int nk = kt + 1 < kt_o ? 4 : nk_last_o;
+            for (int kk = 0; kk < nk; ++kk)
+              mma_bf16_pair(tmem, da0 + soff + 2 * kk, db0 + soff + 2 * kk, ID_O, acc | kk);
+            tc_commit_pair_multicast(&sm.empty[s], 0x3);
+          }
+          __syncwarp();
+          acc = 1;
+          if (++s == P_STAGES) {
+            s = 0;
+            ph ^= 1u;
+            soff = 0;
+          } else {
+            soff += STAGE_DESC;
+          }
+        }
+        for (int kt = 0; kt < kt_j && ok; ++kt) {
+          if (!warp_wait_bounded(&sm.full[s], ph, abort_flag, DEVERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            // scale atoms into the buffer the previous K tile's MMAs do not read
+            const uint32_t sa = tsfa + buf, sb = tsfb + buf;
+            tc_cp_pair_32x128b_warpx4(sa + 0, dsa0 + soff);
+            tc_cp_pair_32x128b_warpx4(sa + 4, dsa0 + soff + 32);
+            tc_cp_pair_32x128b_warpx4(sb + 0, dsb0 + soff);
+            tc_cp_pair_32x128b_warpx4(sb + 8, dsb0 + soff + 32);
+            tc_cp_pair_32x128b_warpx4(sb + 4, dsb0 + soff + 64);
+            tc_cp_pair_32x128b_warpx4(sb + 12, dsb0 + soff + 96);
+            mma_mxf4_pair(tmem, da0 + soff + 0, db0 + soff + 0, ID_J0, sa, sb, acc);
+            mma_mxf4_pair(tmem, da0 + soff + 2, db0 + soff + 2, ID_J2, sa | (2u << 30),
+                          sb | (2u << 30), 1u);
+            mma_mxf4_pair(tmem, da0 + soff + 4, db0 + soff + 4, ID_J0, sa + 4, sb + 8, 1u);
+            mma_mxf4_pair(tmem, da0 + soff + 6, db0 + soff + 6, ID_J2, (sa + 4) | (2u << 30),
+                          (sb + 8) | (2u << 30), 1u);
+            tc_commit_pair_multicast(&sm.empty[s], 0x3);
+          }
+          __syncwarp();
+          acc = 1;
+          buf ^= TMEM_SF_BUF;
+          if (++s == P_STAGES) {
+            s = 0;
+            ph ^= 1u;
+            soff = 0;
+          } else {
+            soff += STAGE_DESC;
+          }
+        }
+        if (!ok) break;
+        if (elect_one()) tc_commit_pair_multicast(&sm.acc_full, 0x3);
+        __syncwarp();
+      }
+      // wait for every MMA / copy issued before tensor memory is freed (the
+      // elected lane is the same one that issued them)
+      if (elect_one()) tc_commit_pair(&sm.drain);
+      __syncwarp();
+      mbar_wait_bounded(&sm.drain, 0u, nullptr, DEVERR_TIMEOUT_MMA);
+      __syncwarp();
+    }
+  } else {
+    // ============================ epilogue (both CTAs) ====================
+    const int ew = warp - 2;
+    const int sp = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(&sm.acc_empty), 0);
+    uint32_t tcount = 0;
+    for (int t = pair; t < ntiles; t += npairs, ++tcount) {
+      int tm, tn;
+      tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
+      int ready = 0;
+      if (lane == 0)
+        ready = mbar_wait_bounded(&sm.acc_full, tcount & 1u, abort_flag, DEVERR_TIMEOUT_EPILOGUE);
+      ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sp) << 16) + 128 * half;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+
+      const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
+      if (row < args.T) {
+        __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = tn * 256 + 128 * half + 32 * c;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = col0 + 8 * q;
+            if (col < args.d_out) {
+              uint32_t p[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                    __uint_as_float(r[c][8 * q + 2 * h]), __uint_as_float(r[c][8 * q + 2 * h + 1]));
+                p[h] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(p[0], p[1], p[2], p[3]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();          // the pair's MMAs, copies and remote arrivals are done
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------
@@ -315,43 +633,93 @@ static PFN_encodeTiled get_encode_fn() {
   return fn;
 }
 
-// 2-D K-major tile map: inner dimension `inner` elements (row stride
-// `row_bytes`), `rows` rows; box = 128 bytes x box_rows with 128-byte swizzle.
+// 2-D tile map: inner dimension `inner` elements (row stride `row_bytes`),
+// `rows` rows; box = `box_inner` elements x `box_rows`.
 static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
-                      uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+                      uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
+                      uint32_t box_inner = 0, bool swizzle128 = true) {
   PFN_encodeTiled enc = get_encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_rows};
+  cuuint32_t box[2] = {box_inner ? box_inner : static_cast<cuuint32_t>(128 / elem_bytes), box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
+size_t gemm_pair_smem_bytes() { return sizeof(PairSmem) + 1024; }
+
+// Number of co-resident CTA pairs of the pair kernel on this device (0 if the
+// query fails); cached per device.
+static int pair_capacity() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] > 0) return cached[dev];
+  const size_t smem = gemm_pair_smem_bytes();
+  if (cudaFuncSetAttribute(gemm_dual_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 148, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel, &cfg) != cudaSuccess || n <= 0)
+    return 0;
+  cached[dev] = n;
+  return n;
+}
+
+// Token counts up to this use the single-CTA kernel (a 256-row pair tile
+// would be mostly padding).
+constexpr int64_t kPairMinT = 129;
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
                         const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
                         void* Y, int64_t ldy, cudaStream_t stream) {
   if (T == 0 || g.d_out == 0) return cudaSuccess;
-  CUtensorMap tm_a, tm_b, tm_ao, tm_bo;
+  const bool pair = T >= kPairMinT && pair_capacity() > 0;
+  const uint32_t brows = pair ? 128 : BN;
+  CUtensorMap tm_a, tm_b, tm_ao, tm_bo, tm_sfa, tm_sfb;
   memset(&tm_a, 0, sizeof(tm_a));
   memset(&tm_b, 0, sizeof(tm_b));
   memset(&tm_ao, 0, sizeof(tm_ao));
   memset(&tm_bo, 0, sizeof(tm_bo));
+  memset(&tm_sfa, 0, sizeof(tm_sfa));
+  memset(&tm_sfb, 0, sizeof(tm_sfb));
   const uint64_t row_j = static_cast<uint64_t>(g.kj_pad / 2);
   if (g.kj_pad > 0) {
     if (!make_tmap(&tm_a, aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, T, row_j, BM) ||
-        !make_tmap(&tm_b, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, g.d_out, row_j, BN))
+        !make_tmap(&tm_b, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, g.d_out, row_j, brows))
       return cudaErrorInvalidValue;
+    if (pair) {
+      // scale buffers seen as rows of 256 bytes; one copy = 4 rows = two 512-byte atoms
+      const uint64_t sfa_rows = static_cast<uint64_t>(round_up(T, kSfaRowPad) * g.nblk / 256);
+      const uint64_t sfb_rows = static_cast<uint64_t>(g.sfb_rows * g.nblk / 256);
+      if (!make_tmap(&tm_sfa, sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfa_rows, 256, 4, 256,
+                     false) ||
+          !make_tmap(&tm_sfb, sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfb_rows, 256, 4, 256,
+                     false))
+        return cudaErrorInvalidValue;
+    }
   }
   if (g.k_pad > 0) {
     const uint64_t row_o = static_cast<uint64_t>(g.k_pad) * 2;
     if (!make_tmap(&tm_ao, xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, T, row_o, BM) ||
-        !make_tmap(&tm_bo, w_hp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, g.d_out, row_o, BN))
+        !make_tmap(&tm_bo, w_hp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, g.d_out, row_o, brows))
       return cudaErrorInvalidValue;
   }
   GemmArgs a;
@@ -365,9 +733,27 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   a.kt_o = static_cast<int>((g.k_pad + 63) / 64);
   a.kt_j = static_cast<int>(g.kj_pad / 256);
   a.k_pad = static_cast<int>(g.k_pad);
-  a.tiles_m = static_cast<int>((T + BM - 1) / BM);
+  a.tiles_m = static_cast<int>((T + (pair ? 255 : BM - 1)) / (pair ? 256 : BM));
   a.tiles_n = static_cast<int>((g.d_out + BN - 1) / BN);
   const int ntiles = a.tiles_m * a.tiles_n;
+  if (pair) {
+    const int npairs = ntiles < pair_capacity() ? ntiles : pair_capacity();
+    const size_t smem = gemm_pair_smem_bytes();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * npairs, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel, tm_a, tm_b, tm_ao, tm_bo, tm_sfa,
+                              tm_sfb, a);
+  }
   const int sms = device_num_sms();
   const int grid = ntiles < sms ? ntiles : sms;
   const size_t smem = gemm_smem_bytes();

@@ -23,7 +23,8 @@
 
 namespace w4a4 {
 
-constexpr int kPrepMaxThreads = 1024;
+constexpr int kPrepMaxConsumers = 512;            // consumer threads per CTA (<= 16 warps)
+constexpr int kPrepMaxThreads = kPrepMaxConsumers + 32;
 
 template <int CH>
 __global__ void __launch_bounds__(kPrepMaxThreads, 1)
@@ -60,16 +61,22 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1)
     // ---------------- producer ----------------
     if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
+      const uint16_t* src = X + static_cast<int64_t>(blockIdx.x) * ldx;
+      const int64_t src_step = static_cast<int64_t>(gridDim.x) * ldx;
       int64_t issued = 0;
+      int s = 0;
+      uint32_t ph = 0;
       for (int64_t i = 0; i < nrows; ++i) {
-        const int s = static_cast<int>(i % stages);
-        const uint32_t ph = static_cast<uint32_t>((i / stages) & 1);
         if (i >= stages && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
           break;
-        const int64_t r = blockIdx.x + i * gridDim.x;
         mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_load(smem + static_cast<size_t>(s) * stage_bytes, X + r * ldx, bytes, &full[s]);
+        bulk_load(smem + static_cast<size_t>(s) * stage_bytes, src, bytes, &full[s]);
+        src += src_step;
         issued = i + 1;
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       if (*abort_flag) {
         // do not leave bulk copies in flight into shared memory we give back
@@ -86,7 +93,7 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1)
   const int ct = threadIdx.x - 32;
   const int rot = (lane >> 3) & 3;
   uint32_t idx[CH][4];     // two 16-bit source columns per register (pair order rotated)
-  float isv[CH][8];
+  float2 isv[CH][4];       // their inv_s
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
     const int chunk = ct + c * NT;
@@ -105,67 +112,99 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1)
         i1 = inv_s[src1];
       }
       idx[c][q] = src0 | (src1 << 16);
-      isv[c][2 * q] = i0;
-      isv[c][2 * q + 1] = i1;
+      isv[c][q] = make_float2(i0, i1);
     }
   }
-  const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
+  // the outlier pair this thread gathers on every row (more pairs than
+  // threads only when k > 2 * NT; those run through the loop below)
   const int xo_row = k_pad >> 1;                            // bf16 pairs per row of X_O
+  uint32_t oidx = static_cast<uint32_t>(d_in) | (static_cast<uint32_t>(d_in) << 16);
+  float2 oinv = make_float2(1.f, 1.f);
+  if (ct < xo_row) {
+    const int o0 = 2 * ct;
+    const uint32_t s0 = o0 < k ? static_cast<uint32_t>(O[o0]) : static_cast<uint32_t>(d_in);
+    const uint32_t s1 = o0 + 1 < k ? static_cast<uint32_t>(O[o0 + 1]) : static_cast<uint32_t>(d_in);
+    oidx = s0 | (s1 << 16);
+    oinv = make_float2(o0 < k ? inv_s[s0] : 1.f, o0 + 1 < k ? inv_s[s1] : 1.f);
+  }
+  const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
+  const int64_t atoms_k = nblk >> 2;
+  const int64_t rstep = gridDim.x;
+  uint8_t* aq_p = aq + static_cast<int64_t>(blockIdx.x) * aq_row;
+  uint32_t* xo_p = xo + static_cast<int64_t>(blockIdx.x) * xo_row;
+  int64_t r = blockIdx.x;
+  int s = 0;
+  uint32_t ph = 0;
 
   for (int64_t i = 0; i < nrows; ++i) {
-    const int s = static_cast<int>(i % stages);
-    const uint32_t ph = static_cast<uint32_t>((i / stages) & 1);
     if (!mbar_wait_bounded(&full[s], ph, abort_flag, DEVERR_TIMEOUT_PREP)) break;
-    const int64_t r = blockIdx.x + i * gridDim.x;
     const uint16_t* row = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(s) * stage_bytes);
+    // scale byte offset of (row r, block 0) in the MMA layout
+    const int64_t sf_row = (((r >> 7) * atoms_k) << 9) + ((r & 31) << 4) + (((r & 127) >> 5) << 2);
 
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int chunk = ct + c * NT;
       if (chunk < nchunks) {                // uniform per warp (nchunks % 32 == 0)
-        float v[8];
+        float2 v[4];
         float amax = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t pr = idx[c][q];
           const float x0 = __uint_as_float(static_cast<uint32_t>(row[pr & 0xFFFFu]) << 16);
           const float x1 = __uint_as_float(static_cast<uint32_t>(row[pr >> 16]) << 16);
-          v[2 * q] = __fmul_rn(x0, isv[c][2 * q]);
-          v[2 * q + 1] = __fmul_rn(x1, isv[c][2 * q + 1]);
-          amax = fmaxf(amax, fmaxf(fabsf(v[2 * q]), fabsf(v[2 * q + 1])));
+          v[q] = __fmul2_rn(make_float2(x0, x1), isv[c][q]);
+          amax = fmaxf(amax, fmaxf(fabsf(v[q].x), fabsf(v[q].y)));
         }
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
         const uint32_t code = mx_scale_code(amax);
         const float inv = mx_inv_scale(code);
-        uint32_t w = cvt_e2m1x8(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv, v[4] * inv,
-                                v[5] * inv, v[6] * inv, v[7] * inv);
+        const float2 inv2 = make_float2(inv, inv);
+        float2 qv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) qv[q] = __fmul2_rn(v[q], inv2);
+        uint32_t w = cvt_e2m1x8(qv[0].x, qv[0].y, qv[1].x, qv[1].y, qv[2].x, qv[2].y, qv[3].x,
+                                qv[3].y);
         w = __funnelshift_l(w, w, 8 * rot);   // undo the pair rotation
-        *reinterpret_cast<uint32_t*>(aq + r * aq_row + 4 * static_cast<int64_t>(chunk)) = w;
+        *reinterpret_cast<uint32_t*>(aq_p + 4 * chunk) = w;
         const uint32_t c4 = __shfl_down_sync(0xFFFFFFFFu, code, 4);
         const uint32_t c8 = __shfl_down_sync(0xFFFFFFFFu, code, 8);
         const uint32_t c12 = __shfl_down_sync(0xFFFFFFFFu, code, 12);
         if ((lane & 15) == 0) {
-          const int64_t kb = chunk >> 2;       // multiple of 4
-          *reinterpret_cast<uint32_t*>(sfa + sf_offset(r, kb, nblk)) =
+          // blocks chunk/4 .. chunk/4 + 3 of row r: one 4-byte word of an atom
+          *reinterpret_cast<uint32_t*>(sfa + sf_row + ((static_cast<int64_t>(chunk) >> 4) << 9)) =
               code | (c4 << 8) | (c8 << 16) | (c12 << 24);
         }
       }
     }
-    for (int i2 = ct; i2 < xo_row; i2 += NT) {
-      const int o0 = 2 * i2;
-      const int src0 = o0 < k ? O[o0] : d_in;
-      const int src1 = o0 + 1 < k ? O[o0 + 1] : d_in;
-      const float s0 = o0 < k ? inv_s[src0] : 1.f;
-      const float s1 = o0 + 1 < k ? inv_s[src1] : 1.f;
-      const float v0 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src0]) << 16), s0);
-      const float v1 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src1]) << 16), s1);
-      const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(v0));
-      const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(v1));
-      xo[r * xo_row + i2] = b0 | (b1 << 16);
+    if (ct < xo_row) {
+      const float x0 = __uint_as_float(static_cast<uint32_t>(row[oidx & 0xFFFFu]) << 16);
+      const float x1 = __uint_as_float(static_cast<uint32_t>(row[oidx >> 16]) << 16);
+      const float2 v = __fmul2_rn(make_float2(x0, x1), oinv);
+      xo_p[ct] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                 (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+      for (int i2 = ct + NT; i2 < xo_row; i2 += NT) {
+        const int o0 = 2 * i2;
+        const int src0 = o0 < k ? O[o0] : d_in;
+        const int src1 = o0 + 1 < k ? O[o0 + 1] : d_in;
+        const float y0 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src0]) << 16),
+                                   o0 < k ? inv_s[src0] : 1.f);
+        const float y1 = __fmul_rn(__uint_as_float(static_cast<uint32_t>(row[src1]) << 16),
+                                   o0 + 1 < k ? inv_s[src1] : 1.f);
+        xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
+                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    r += rstep;
+    aq_p += rstep * aq_row;
+    xo_p += rstep * xo_row;
   }
 }
 
@@ -177,9 +216,8 @@ struct PrepPlan {
 static PrepPlan plan_prep(const Geometry& g) {
   PrepPlan p{};
   const int nchunks = static_cast<int>(g.kj_pad / 8);
-  const int max_nt = kPrepMaxThreads - 32;
   p.ch = 1;
-  while (p.ch < 4 && (nchunks + p.ch - 1) / p.ch > max_nt) p.ch *= 2;
+  while (p.ch < 8 && (nchunks + p.ch - 1) / p.ch > kPrepMaxConsumers) p.ch *= 2;
   int nt = (nchunks + p.ch - 1) / p.ch;
   nt = static_cast<int>(round_up(nt < 32 ? 32 : nt, 32));
   p.nt = nt;
@@ -193,7 +231,7 @@ static PrepPlan plan_prep(const Geometry& g) {
 bool prep_supported(const Geometry& g) {
   if (g.d_in > 65535) return false;
   const int nchunks = static_cast<int>(g.kj_pad / 8);
-  if (nchunks > 4 * (kPrepMaxThreads - 32)) return false;
+  if (nchunks > 8 * kPrepMaxConsumers) return false;
   return plan_prep(g).smem <= 227 * 1024;
 }
 
@@ -223,7 +261,8 @@ cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_
   switch (p.ch) {
     case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
     case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
-    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+    case 4: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+    default: return launch_prep_ch<8>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
   }
 }
 

@@ -47,7 +47,8 @@ typedef enum w4a4_status {
   W4A4_ERR_INVALID_ARG = 1,      /* null pointer, negative size, alpha outside (0,1), k > d_in */
   W4A4_ERR_UNSUPPORTED_SHAPE = 2,/* alignment or size outside the supported set above */
   W4A4_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
-  W4A4_ERR_TIMEOUT = 4           /* a device pipeline wait ran out (see w4a4_last_error) */
+  W4A4_ERR_TIMEOUT = 4,          /* a device pipeline wait ran out (see w4a4_last_error) */
+  W4A4_ERR_SCRATCH_LIMIT = 5     /* the problem needs more scratch than w4a4_linear_noalloc has */
 } w4a4_status;
 
 /* Weight scale layouts of the block packing (review sec. 3.4: "32x32 tiles"
@@ -193,6 +194,36 @@ w4a4_status w4a4_linear(const void* X, int64_t T, int64_t ldx, const w4a4_packed
 w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_weight* pw,
                              void* X_dev, void* workspace, size_t ws_bytes, void* Y_dev,
                              void* Y_host, void* stream);
+
+/* Size of the fixed device scratch array behind w4a4_linear_noalloc. */
+#define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* The online layer (w4a4_prep_act then w4a4_gemm_dual, exactly as
+ * w4a4_linear) without a caller workspace and without allocating anything.
+ * The paper has no counterpart to this call: it is a service for callers that
+ * cannot hand the library device memory at the point where the layer runs --
+ * a host framework or plugin that owns every device allocation and passes
+ * only inputs and outputs, or a serving loop whose device memory is fixed at
+ * start-up, where allocating (and the synchronisation cudaMalloc / cudaFree
+ * may imply) is not allowed per call.
+ *   Scratch: a static device array of W4A4_NOALLOC_SCRATCH_BYTES (32 MiB) in
+ *   the library, held on every device the library is used on until the
+ *   process exits.  A problem whose w4a4_workspace_size exceeds it returns
+ *   W4A4_ERR_SCRATCH_LIMIT before anything is enqueued (at d_in = 5120,
+ *   k = 32 about 12000 tokens fit; use w4a4_linear for larger T).
+ *   Sharing: every call on a device uses the same array, which keeps what the
+ *   previous call left there.  No byte needs clearing -- the scale rows past T
+ *   that a call reads without writing reach only output rows past T, which
+ *   are never stored -- but calls whose GPU work overlaps (other streams,
+ *   other host threads) race on the array and must be serialised by the
+ *   caller.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (a host-side query, with that device current; nothing is allocated).
+ *   Make that first call before any stream capture.
+ * Arguments, layouts and the other errors are those of w4a4_linear. */
+w4a4_status w4a4_linear_noalloc(const void* X, int64_t T, int64_t ldx,
+                                const w4a4_packed_weight* pw, void* Y, int64_t ldy,
+                                void* stream);
 
 /* Synchronises `stream` and reports device-side failures recorded since the
  * last clear: W4A4_OK, or W4A4_ERR_TIMEOUT if a bounded wait ran out (the

@@ -104,3 +104,25 @@ def test_calib_validation():
     assert w4._calib_finalize(f, f, 64, 0.5, 65, f, f, f, f, f, None) == w4.ERR_INVALID_ARG  # k > d_in
     assert w4._calib_finalize(f, f, 64, 0.5, 4, f, f, f, None, f, None) == w4.ERR_INVALID_ARG  # O missing
     assert w4._calib_finalize(f, f, 20000, 0.5, 4, f, f, f, f, f, None) == w4.ERR_UNSUPPORTED_SHAPE
+
+
+def test_noalloc_limit_and_validation_before_launch():
+    # the scratch limit in the header is the one the binding reports
+    hdr = open(os.path.join(ROOT, "include", "w4a4.h")).read()
+    m = re.search(r"#define W4A4_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m and int(m.group(1)) << int(m.group(2)) == w4.NOALLOC_SCRATCH_BYTES
+    assert "no-alloc scratch" in w4.status_string(w4.ERR_SCRATCH_LIMIT)
+    # about 12000 tokens of a 5120-wide layer with 32 outliers fit, 12100 do not
+    assert w4.workspace_size(12000, 5120, 13824, 32) <= w4.NOALLOC_SCRATCH_BYTES
+    assert w4.workspace_size(12100, 5120, 13824, 32) > w4.NOALLOC_SCRATCH_BYTES
+    # Pointers here are never dereferenced: each call returns before any CUDA work.
+    pw = _raw_pw()
+    f = 0x1000
+    assert w4._linear_noalloc(f, 8, 63, ctypes.byref(pw), f, 32, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_noalloc(f, 8, 64, ctypes.byref(pw), f, 31, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_noalloc(None, 8, 64, ctypes.byref(pw), f, 32, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_noalloc(f, -1, 64, ctypes.byref(pw), f, 32, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_noalloc(f, 0, 64, ctypes.byref(pw), f, 32, None) == w4.OK
+    assert w4._linear_noalloc(f, 1 << 20, 64, ctypes.byref(pw), f, 32, None) \
+        == w4.ERR_SCRATCH_LIMIT
+

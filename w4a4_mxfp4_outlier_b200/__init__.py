@@ -21,10 +21,11 @@ LIB_PATH = os.path.join(_HERE, "libw4a4.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libw4a4.so is not built ({LIB_PATH}); run "
-                      "`python -m w4a4_mxfp4_outlier_b200.build`")
+                      "`python w4a4_mxfp4_outlier_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(6)
+NOALLOC_SCRATCH_BYTES = 32 << 20     # W4A4_NOALLOC_SCRATCH_BYTES
 SF_32x1_KMAJOR, SF_32x32_TILE = 0, 1
 
 _i64 = ctypes.c_int64
@@ -72,13 +73,15 @@ _linear = _sig("w4a4_linear", _st, _vp, _i64, _i64, ctypes.POINTER(PackedWeightC
                ctypes.c_size_t, _vp, _i64, _vp)
 _linear_host = _sig("w4a4_linear_host", _st, _vp, _i64, ctypes.POINTER(PackedWeightC), _vp, _vp,
                     ctypes.c_size_t, _vp, _vp, _vp)
+_linear_noalloc = _sig("w4a4_linear_noalloc", _st, _vp, _i64, _i64, ctypes.POINTER(PackedWeightC),
+                       _vp, _i64, _vp)
 _last_error = _sig("w4a4_last_error", _st, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32))
 
 EXPORTED = [
     "w4a4_abi_version", "w4a4_status_string", "w4a4_num_sms", "w4a4_get_dims",
     "w4a4_calib_observe", "w4a4_calib_finalize", "w4a4_weight_sizes", "w4a4_pack_weight",
     "w4a4_workspace_size", "w4a4_prep_act", "w4a4_gemm_dual", "w4a4_linear",
-    "w4a4_linear_host", "w4a4_last_error",
+    "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
 ]
 
 
@@ -260,6 +263,17 @@ def linear_host(X_host: torch.Tensor, pw: PackedWeight, X_dev: torch.Tensor, wor
     _check(_linear_host(_ptr(X_host), X_host.shape[0], ctypes.byref(c), _ptr(X_dev),
                         _ptr(workspace), workspace.numel() * workspace.element_size(),
                         _ptr(Y_dev), _ptr(Y_host), _stream(stream)), "linear_host")
+
+
+def linear_noalloc(X: torch.Tensor, pw: PackedWeight, Y: torch.Tensor, stream=None):
+    """The online layer with the library's fixed scratch array instead of a
+    workspace: allocates nothing, for callers that cannot hand over device
+    memory.  Problems larger than NOALLOC_SCRATCH_BYTES of workspace raise
+    W4A4Error(ERR_SCRATCH_LIMIT); calls overlapping on the GPU must be
+    serialised by the caller (they share the array)."""
+    c = pw.c
+    _check(_linear_noalloc(_ptr(X), X.shape[0], X.stride(0), ctypes.byref(c), _ptr(Y), Y.stride(0),
+                           _stream(stream)), "linear_noalloc")
 
 
 def last_error(clear: bool = True, stream=None):

@@ -1,6 +1,9 @@
 """Build libw4a4.so in-tree with nvcc for sm_100a.
 
-    python -m w4a4_mxfp4_outlier_b200.build [--force]
+    python w4a4_mxfp4_outlier_b200/build.py [--force] [-v]
+
+(run as a script, not as a module of the package: importing the package loads
+the library this builds)
 
 csrc/libw4a4.cu (which includes every kernel file and the C-ABI) is compiled
 as one translation unit and linked into one shared library next to this file.  The CUDA
@@ -21,7 +24,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["libw4a4.cu"]
 HEADERS = ["w4a4_device.cuh", "w4a4_internal.h", "w4a4_api.cu", "calib.cu", "prep.cu",
-           "pack.cu", "gemm.cu"]
+           "pack.cu", "gemm.cu", "noalloc.cu"]
 
 
 def nvcc() -> str:

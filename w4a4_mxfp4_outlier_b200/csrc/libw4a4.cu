@@ -6,3 +6,4 @@
 #include "pack.cu"
 #include "prep.cu"
 #include "gemm.cu"
+#include "noalloc.cu"

@@ -75,6 +75,7 @@ const char* w4a4_status_string(w4a4_status s) {
     case W4A4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or alignment";
     case W4A4_ERR_CUDA: return "CUDA error";
     case W4A4_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case W4A4_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed no-alloc scratch";
   }
   return "unknown status";
 }

@@ -104,77 +104,130 @@ __global__ void finalize_scales_kernel(const float* __restrict__ act, const floa
   score[j] = __fmul_rn(act[j], ij);
 }
 
-// Step 2 (one block): order the columns by (score descending, index
-// ascending) with a bitonic sort of 64-bit keys in shared memory, flag the
-// first k as outliers, then compact the flags into O and jmap (both
-// ascending).  Keys: high word 0xFFFFFFFF - score bits (non-negative floats
-// order like their bit patterns), low word the column index; padding keys
-// are all-ones and sort last.
+// Step 2 (one block): select the k columns of largest (score, -index) --
+// score descending, lower index first among equal scores -- then compact the
+// selection into O and the rest into jmap (both ascending).
+//
+// Selection is a radix select on a 48-bit key per column, 8 bits per pass
+// from the top: key = score bits << 16 | (0xFFFF - index).  Non-negative
+// floats order like their bit patterns and the low field breaks ties towards
+// the lower index, so keys are distinct and the k largest keys are exactly the
+// k columns wanted.  Each pass histograms the candidates that still match the
+// prefix found so far, and one warp picks the digit holding the k-th largest
+// key.  Thread t owns the contiguous columns [t*per, (t+1)*per), which keeps
+// the final compaction in index order with one block-wide scan.
 constexpr int kFinalizeMaxD = 16384;
 constexpr int kFinalizeThreads = 1024;
+constexpr int kFinalizePer = kFinalizeMaxD / kFinalizeThreads;   // columns per thread, at most
 
 __global__ void __launch_bounds__(kFinalizeThreads)
     finalize_select_kernel(const float* __restrict__ score, int d_in, int k,
                            int32_t* __restrict__ O, int32_t* __restrict__ jmap) {
-  extern __shared__ __align__(16) uint8_t fsmem[];
-  uint64_t* key = reinterpret_cast<uint64_t*>(fsmem);                  // [n]
-  int* cnt = reinterpret_cast<int*>(fsmem + kFinalizeMaxD * 8);         // [1024]
-  uint8_t* flag = fsmem + kFinalizeMaxD * 8 + kFinalizeThreads * 4;     // [d_in]
-  int n = 1;
-  while (n < d_in) n <<= 1;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    if (i < d_in) {
-      const uint32_t b = __float_as_uint(score[i]);
-      key[i] = (static_cast<uint64_t>(0xFFFFFFFFu - b) << 32) | static_cast<uint32_t>(i);
-      flag[i] = 0;
-    } else {
-      key[i] = ~0ull;
-    }
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t warp_cnt[kFinalizeThreads / 32];
+  __shared__ uint64_t sel_prefix;
+  __shared__ uint32_t sel_remaining;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int per = (d_in + kFinalizeThreads - 1) / kFinalizeThreads;
+  const int lo = tid * per < d_in ? tid * per : d_in;
+  const int hi = lo + per < d_in ? lo + per : d_in;
+
+  uint64_t key[kFinalizePer];
+#pragma unroll
+  for (int e = 0; e < kFinalizePer; ++e) {
+    const int j = lo + e;
+    key[e] = j < hi ? (static_cast<uint64_t>(__float_as_uint(score[j])) << 16) |
+                          static_cast<uint64_t>(0xFFFFu - static_cast<uint32_t>(j))
+                    : 0ull;
   }
-  __syncthreads();
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
-        const int i = 2 * t - (t & (stride - 1));      // lower element of the pair
-        const int j = i + stride;
-        const bool up = (i & size) == 0;
-        const uint64_t a = key[i], b = key[j];
-        if ((a > b) == up) {
-          key[i] = b;
-          key[j] = a;
+
+  // threshold = the k-th largest key (keys are distinct); selected: key >= threshold
+  uint64_t thr = ~0ull;                    // k == 0: nothing reaches it
+  if (k > 0) {
+    if (tid == 0) {
+      sel_prefix = 0;
+      sel_remaining = static_cast<uint32_t>(k);
+    }
+    for (int shift = 40; shift >= 0; shift -= 8) {
+      for (int b = tid; b < 256; b += kFinalizeThreads) hist[b] = 0;
+      __syncthreads();
+      const uint64_t prefix = sel_prefix;
+      const uint64_t above = shift + 8 < 64 ? ~0ull << (shift + 8) : 0ull;
+#pragma unroll
+      for (int e = 0; e < kFinalizePer; ++e)
+        if (lo + e < hi && (key[e] & above) == prefix)
+          atomicAdd(&hist[(key[e] >> shift) & 0xFFu], 1u);
+      __syncthreads();
+      if (warp == 0) {
+        // lane l covers digits 8l .. 8l+7; count the candidates above each lane's range
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          c[q] = hist[8 * lane + q];
+          sum += c[q];
+        }
+        uint32_t incl = sum;                 // inclusive suffix sum over lanes l..31
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, off);
+          if (lane + off < 32) incl += v;
+        }
+        const uint32_t rem = sel_remaining;
+        uint32_t acc = incl - sum;           // candidates with a digit above this lane's range
+        if (acc < rem && rem <= incl) {      // exactly one lane
+          int d = 7;
+          while (d > 0 && acc + c[d] < rem) {
+            acc += c[d];
+            --d;
+          }
+          sel_prefix = prefix | (static_cast<uint64_t>(8 * lane + d) << shift);
+          sel_remaining = rem - acc;
         }
       }
       __syncthreads();
     }
+    thr = sel_prefix;
   }
-  for (int r = threadIdx.x; r < k; r += blockDim.x) flag[static_cast<uint32_t>(key[r])] = 1;
-  __syncthreads();
-  const int per = (d_in + kFinalizeThreads - 1) / kFinalizeThreads;
-  const int lo = threadIdx.x * per < d_in ? threadIdx.x * per : d_in;
-  const int hi = lo + per < d_in ? lo + per : d_in;
-  int c = 0;
-  for (int j = lo; j < hi; ++j) c += flag[j];
-  cnt[threadIdx.x] = c;
-  __syncthreads();
-  for (int off = 1; off < kFinalizeThreads; off <<= 1) {     // inclusive scan
-    const int v = threadIdx.x >= off ? cnt[threadIdx.x - off] : 0;
-    __syncthreads();
-    cnt[threadIdx.x] += v;
-    __syncthreads();
+
+  // compaction in index order
+  uint32_t flags = 0, c = 0;
+#pragma unroll
+  for (int e = 0; e < kFinalizePer; ++e)
+    if (lo + e < hi && key[e] >= thr) {
+      flags |= 1u << e;
+      ++c;
+    }
+  uint32_t incl = c;                         // inclusive scan over the warp
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
   }
-  int o = cnt[threadIdx.x] - c;          // outliers before this run
-  int jj = lo - o;                       // kept columns before this run
-  for (int j = lo; j < hi; ++j) {
-    if (flag[j]) {
-      O[o++] = j;
-    } else {
-      jmap[jj++] = j;
+  if (lane == 31) warp_cnt[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = warp_cnt[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, w, off);
+      if (lane >= off) w += v;
+    }
+    warp_cnt[lane] = w;                      // inclusive over warps
+  }
+  __syncthreads();
+  int o = static_cast<int>(incl - c + (warp > 0 ? warp_cnt[warp - 1] : 0u));   // outliers before lo
+  int jj = lo - o;                                                               // kept columns before lo
+#pragma unroll
+  for (int e = 0; e < kFinalizePer; ++e) {
+    const int j = lo + e;
+    if (j < hi) {
+      if ((flags >> e) & 1u)
+        O[o++] = j;
+      else
+        jmap[jj++] = j;
     }
   }
-}
-
-size_t finalize_smem_bytes() {
-  return static_cast<size_t>(kFinalizeMaxD) * 8 + kFinalizeThreads * 4 + kFinalizeMaxD;
 }
 
 int finalize_max_d() { return kFinalizeMaxD; }
@@ -186,11 +239,7 @@ cudaError_t launch_finalize(const float* act, const float* wsc, int d_in, double
   finalize_scales_kernel<<<nb, 256, 0, stream>>>(act, wsc, d_in, alpha, s, inv_s, score);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = finalize_smem_bytes();
-  e = cudaFuncSetAttribute(finalize_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  finalize_select_kernel<<<1, kFinalizeThreads, smem, stream>>>(score, d_in, k, O, jmap);
+  finalize_select_kernel<<<1, kFinalizeThreads, 0, stream>>>(score, d_in, k, O, jmap);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@
  *  - Arguments are validated before anything is launched.  On a non-OK
  *    return nothing was enqueued and outputs are untouched.
  *  - Supported shapes: d_in % 8 == 0, d_out % 16 == 0, row strides % 8 == 0,
- *    all pointers 16-byte aligned, kj_pad <= 31744 (see w4a4_dims).
+ *    all pointers 16-byte aligned, d_in <= 16384.
  *    Anything else returns W4A4_ERR_UNSUPPORTED_SHAPE.
  *  - Device-side failures (a pipeline wait that runs out, about 2 s) are
  *    recorded in a device error word; w4a4_last_error() reads it.  No kernel

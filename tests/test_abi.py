@@ -126,3 +126,10 @@ def test_noalloc_limit_and_validation_before_launch():
     assert w4._linear_noalloc(f, 1 << 20, 64, ctypes.byref(pw), f, 32, None) \
         == w4.ERR_SCRATCH_LIMIT
 
+
+def test_prep_width_limit():
+    # activation prep stages whole rows of at most 16384 bf16 in shared memory
+    pw = _raw_pw(d_in=16392, d_out=32, k=4)
+    assert w4._prep_act(0x1000, 8, 16392, ctypes.byref(pw), 0x1000, 0x1000, 0x1000, None) \
+        == w4.ERR_UNSUPPORTED_SHAPE
+

@@ -178,6 +178,31 @@ class ClockSampler:
                 "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
+# gemm_dual_pair_kernel on the "full" workload (mean of the up and down
+# launches), from one ncu capture of this bench (summary and command in
+# profiles/gemm_dual_pair_traffic_full_T57600.md).  Valid only for the GEMM
+# sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
+# for any other source or workload.
+GEMM_TRAFFIC = {
+    "sha256": "392bb6a4ca7679722ed6fb15ce83149887ed331b22eea44e0fe922733e2b5345",
+    "workload": "full",
+    "bytes_per_launch": (728140288 + 1555996928 + 1510572032 + 571407872) / 2,
+}
+
+
+def gemm_traffic(workload: str):
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "w4a4_mxfp4_outlier_b200", "csrc")
+    for f in ("gemm.cu", "w4a4_device.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != GEMM_TRAFFIC["sha256"] or workload != GEMM_TRAFFIC["workload"]:
+        return None
+    return int(GEMM_TRAFFIC["bytes_per_launch"])
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -314,7 +339,8 @@ def run_gpu(args):
     other = peaks["bf16_tflops_sustained" if boost else "bf16_tflops"] * FP4_PER_BF16
     roof = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
-            "traffic": None,
+            "traffic": gemm_traffic(args.workload),
+            "traffic_unit": "bytes per launch (ncu dram read + write)",
             "kernel": "gemm_dual_pair_kernel",
             "peak_source": f"{src}: {key} x {FP4_PER_BF16:g} (nominal FP4:BF16 ratio), of measured",
             "frac_of_other_peak": round(gemm_tflops / other, 4),
@@ -498,7 +524,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="full",
-                    choices=["full", "full_up", "full_down", "mid_up", "ffn0", "ffn2", "tiny", "sweep"])
+                    choices=["full", "full_up", "full_down", "mid_up", "mid_down", "ffn0", "ffn2", "tiny",
+                             "sweep"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -116,6 +116,7 @@ def sweep_layers():
 
 
 MID_UP = Layer("mid_up_T16384", 16384, 5120, 13824, 0.6, 32, 0, X_UP, W_UP)
+MID_DOWN = FULL_DOWN.with_(name="mid_down_T16384", T=16384)
 
 WORKLOADS = {
     "tiny": [TINY],
@@ -125,6 +126,7 @@ WORKLOADS = {
     "full_up": [FULL_UP],
     "full_down": [FULL_DOWN],
     "mid_up": [MID_UP],
+    "mid_down": [MID_DOWN],
     "sweep": sweep_layers(),
 }
 

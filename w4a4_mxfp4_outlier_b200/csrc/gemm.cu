@@ -332,8 +332,11 @@ constexpr int P_SFB_BYTES = 2048;             // all 256 output rows x 8 blocks
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;
 constexpr int P_EPI_ARRIVALS = 2 * NUM_EPI_WARPS;
 
+constexpr int P_EPI_BYTES = 16 * 64;          // staging block: 16 rows x 32 bf16 (64-byte swizzle)
+
 struct PairSmem {
   uint8_t stage[P_STAGES][P_STAGE_BYTES];
+  alignas(1024) uint8_t epi[NUM_EPI_WARPS][P_EPI_BYTES];   // per epilogue warp: Y staging
   uint64_t full[P_STAGES];     // leader's counts the bytes of both CTAs
   uint64_t empty[P_STAGES];    // both CTAs: MMA commit, multicast
   uint64_t acc_full;           // both CTAs: MMA commit, multicast
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
-                          const GemmArgs args) {
+                          const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   PairSmem& sm = *reinterpret_cast<PairSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -576,29 +579,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
-      const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
-      if (row < args.T) {
-        __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
+      // Y through a per-warp staging block, 16 rows x 32 columns at a time:
+      // the lanes holding those rows write them (64-byte swizzle: 16-byte
+      // chunk j of row r sits at chunk j ^ ((r >> 1) & 3), so the writes hit
+      // distinct banks) and one lane stores the block with a TMA tile store,
+      // which also clips rows past T and columns past d_out.
+      const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp;
+      const uint32_t stg = smem_u32(sm.epi[ew]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col0 = tn * 256 + 128 * half + 32 * c;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t p[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = col0 + 8 * q;
-            if (col < args.d_out) {
-              uint32_t p[4];
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[c][2 * j]),
+                                                          __uint_as_float(r[c][2 * j + 1]));
+          p[j] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        const int col = tn * 256 + 128 * half + 32 * c;
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                    __uint_as_float(r[c][8 * q + 2 * h]), __uint_as_float(r[c][8 * q + 2 * h + 1]));
-                p[h] = *reinterpret_cast<const uint32_t*>(&b2);
-              }
-              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(p[0], p[1], p[2], p[3]);
-            }
+        for (int hh = 0; hh < 2; ++hh) {
+          // the previous store from this block must have read it
+          if (elect_one()) bulk_wait_group_read0();
+          __syncwarp();
+          if ((lane >> 4) == hh) {
+            const uint32_t rl = static_cast<uint32_t>(lane & 15);
+            const uint32_t dst = stg + rl * 64u;
+#pragma unroll
+            for (uint32_t q = 0; q < 4; ++q)
+              st_shared_v4(dst + 16u * (q ^ ((rl >> 1) & 3u)), p[4 * q], p[4 * q + 1], p[4 * q + 2],
+                           p[4 * q + 3]);
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (elect_one()) {
+            tma_store_2d(&tm_y, stg, col, row0 + 16 * hh);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
       }
     }
+    if (elect_one()) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -637,7 +659,8 @@ static PFN_encodeTiled get_encode_fn() {
 // `rows` rows; box = `box_inner` elements x `box_rows`.
 static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                       uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
-                      uint32_t box_inner = 0, bool swizzle128 = true) {
+                      uint32_t box_inner = 0, bool swizzle128 = true,
+                      CUtensorMapSwizzle swz_other = CU_TENSOR_MAP_SWIZZLE_NONE) {
   PFN_encodeTiled enc = get_encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -646,7 +669,7 @@ static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : swz_other,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -751,8 +774,14 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // Y as bf16 tiles of 16 rows x 32 columns, 64-byte swizzle (epilogue staging layout)
+    CUtensorMap tm_y;
+    memset(&tm_y, 0, sizeof(tm_y));
+    if (!make_tmap(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
+                   static_cast<uint64_t>(ldy) * 2, 16, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
     return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel, tm_a, tm_b, tm_ao, tm_bo, tm_sfa,
-                              tm_sfb, a);
+                              tm_sfb, tm_y, a);
   }
   const int sms = device_num_sms();
   const int grid = ntiles < sms ? ntiles : sms;

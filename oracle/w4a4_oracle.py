@@ -62,6 +62,7 @@ E8M0_BIAS = 127
 
 LAYOUT_32x1 = 0        # one scale per 32 consecutive K of one output row
 LAYOUT_32x32 = 1       # one scale per 32 (rows) x 32 (K) tile
+LAYOUT_128x1 = 2       # one scale per 128 consecutive K of one output row (4 MX blocks)
 
 
 # ----------------------------------------------------------------------------
@@ -282,11 +283,12 @@ def pack_weight(W: np.ndarray, s: np.ndarray, O: np.ndarray, J: np.ndarray,
     W: float32 values [d_out, d_in] (bf16-exact).  Returns a dict with
       wq    uint8 [d_out, nblk*16]  packed codes of the compacted J columns
       sfb   uint8 [d_out, nblk]     E8M0 codes (32x32: the tile's code repeated
-                                    on each of its 32 rows)
+                                    on each of its 32 rows; 128x1: the stripe's
+                                    code repeated on its 4 blocks)
       w_hp  uint16 [d_out, k]       bfloat16 bits of the folded O columns
     Rows are processed in chunks (a multiple of 32) only to bound memory.
     """
-    if layout not in (LAYOUT_32x1, LAYOUT_32x32):
+    if layout not in (LAYOUT_32x1, LAYOUT_32x32, LAYOUT_128x1):
         raise ValueError("unknown layout")
     d_out = W.shape[0]
     kj = J.shape[0]
@@ -304,6 +306,16 @@ def pack_weight(W: np.ndarray, s: np.ndarray, O: np.ndarray, J: np.ndarray,
         WJ = _pad_cols(Wf[:, J], nb * MX_BLOCK).reshape(r1 - r0, nb, MX_BLOCK)
         if layout == LAYOUT_32x1:
             sc, codes = mxfp4_quantize_blocks(WJ)
+        elif layout == LAYOUT_128x1:
+            # [review §3.4] "128x1 K-major stripe": one amax per 128 consecutive
+            # compacted K of a row, i.e. per 4 consecutive MX blocks from p = 0;
+            # a last partial stripe is completed with zero blocks
+            amax_blocks = np.max(np.abs(WJ), axis=-1)                        # [rows, nb]
+            padb = (-nb) % 4
+            amax_blocks = np.concatenate(
+                [amax_blocks, np.zeros((r1 - r0, padb), np.float32)], axis=1)
+            stripe = amax_blocks.reshape(r1 - r0, -1, 4).max(axis=-1)        # [rows, stripes]
+            sc, codes = mxfp4_quantize_blocks(WJ, np.repeat(stripe, 4, axis=1)[:, :nb])
         else:
             # one amax per 32 rows x 32 columns; rows past d_out count as zeros
             amax_rows = np.max(np.abs(WJ), axis=-1)                          # [rows, nb]

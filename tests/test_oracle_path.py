@@ -219,6 +219,64 @@ def test_32x32_tiles_share_one_scale():
     assert int(sfb[0, 0]) == int(orc.mx_shared_exponent(np.array([amax]))[0]) + 127
 
 
+def _pack_plain(W, layout):
+    """pack_weight with s = 1, no outliers: plain per-row encoding of W."""
+    d_in = W.shape[1]
+    return orc.pack_weight(W.astype(np.float32), np.ones(d_in, np.float32),
+                           np.zeros(0, np.int64), np.arange(d_in), layout)
+
+
+def test_128x1_stripe_hand_worked():
+    """[review §3.4] 128x1 K-major stripe: 4 consecutive MX blocks of a row
+    share the exponent of the stripe's largest element (values worked by hand
+    on the E2M1 grid)."""
+    W = np.zeros((1, 256), np.float32)
+    W[0, 0] = 6.0                                        # stripe 0 amax 6 -> e = 0
+    W[0, 32:37] = [0.25, 0.75, -2.5, 0.09375, 1.5]       # block 1, coded with e = 0
+    W[0, 160] = 0.09375                                  # stripe 1 amax 3/32 -> e = -6
+    p = _pack_plain(W, orc.LAYOUT_128x1)
+    assert p["sfb"][0].tolist() == [127] * 4 + [121] * 4
+    codes = orc.unpack_nibbles(p["wq"])[0]
+    assert codes[0] == 0x7                               # 6
+    assert codes[32:37].tolist() == [0x0, 0x2, 0xC, 0x0, 0x3]   # 0.25->0 (tie), 0.75->1, -2.5->-2 (tie), 3/32->0, 1.5
+    assert codes[160] == 0x7                             # 3/32 * 64 = 6
+    # the 32x1 layout gives block 1 its own exponent: amax 2.5 -> e = -1
+    q = _pack_plain(W, orc.LAYOUT_32x1)
+    assert q["sfb"][0, 1] == 126 and q["sfb"][0, 0] == 127 and q["sfb"][0, 5] == 121
+
+
+def test_128x1_equals_32x1_when_blocks_share_amax():
+    """If the 4 blocks of every stripe have the same amax, sharing it changes
+    nothing: the 128x1 packing equals the 32x1 packing."""
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((40, 512)) * 0.3).astype(np.float32)
+    W = np.clip(W, -1.0, 1.0)
+    W[:, ::32] = 1.5 * np.sign(W[:, ::32] + 0.5)         # every block holds +-1.5 as its max
+    a = _pack_plain(W, orc.LAYOUT_128x1)
+    b = _pack_plain(W, orc.LAYOUT_32x1)
+    np.testing.assert_array_equal(a["sfb"], b["sfb"])
+    np.testing.assert_array_equal(a["wq"], b["wq"])
+
+
+def test_128x1_stripes_share_scale_and_saturate_at_max():
+    X, W = _small(T=8, d_in=600, d_out=48)
+    _, p = orc.linear_reference(X, W, 0.6, 7, layout=orc.LAYOUT_128x1)
+    sfb = p["sfb"]
+    nb = sfb.shape[1]
+    for b0 in range(0, nb, 4):
+        st = sfb[:, b0:b0 + 4]
+        assert np.all(st == st[:, 0:1])
+    # the stripe maximum codes to magnitude 6 or 7 (|q| in [4, 8))
+    codes = orc.unpack_nibbles(p["wq"]) & 0x7
+    Vw = orc.fold_weight(W.astype(np.float32), p["s"])[:, p["J"]]
+    for r in range(48):
+        for b0 in range(0, nb, 4):
+            seg = np.abs(Vw[r, b0 * 32:(b0 + 4) * 32])
+            if seg.size and seg.max() > 0:
+                i = b0 * 32 + int(np.argmax(seg))
+                assert codes[r, i] in (6, 7)
+
+
 def test_tiny_generator_matches_pages_statistics():
     """The tiny workload's planted channels exceed 6.0, weights stay below 0.6
     (review §3.1), and after smoothing the planted channels are the top-8."""

@@ -52,10 +52,13 @@ typedef enum w4a4_status {
 } w4a4_status;
 
 /* Weight scale layouts of the block packing (review sec. 3.4: "32x32 tiles"
- * and K-major stripes; the stripe is 32x1 here, the MXFP4 block length). */
+ * and "128x1 K-major stripes"; 32x1 is the plain MXFP4 block).  All three
+ * are stored in the same per-block MMA layout, so the GEMM reads them alike. */
 typedef enum w4a4_wlayout {
   W4A4_SF_32x1_KMAJOR = 0,  /* one E8M0 per 32 consecutive compacted K of one output row */
-  W4A4_SF_32x32_TILE = 1    /* one E8M0 per 32 output rows x 32 compacted K, stored on each row */
+  W4A4_SF_32x32_TILE = 1,   /* one E8M0 per 32 output rows x 32 compacted K, stored on each row */
+  W4A4_SF_128x1_KMAJOR = 2  /* one E8M0 per 128 consecutive compacted K of one output row,
+                               stored on each of its 4 blocks */
 } w4a4_wlayout;
 
 int w4a4_abi_version(void);

@@ -77,7 +77,7 @@ class Layer:
     d_out: int
     alpha: float
     k: int
-    layout: int          # 0 = 32x1 K-major scale stripes, 1 = 32x32 tiles
+    layout: int          # 0 = 32x1 K-major scale stripes, 1 = 32x32 tiles, 2 = 128x1 stripes
     x: XSpec
     w: WSpec
     seed: int = 0
@@ -105,10 +105,11 @@ FULL_DOWN = Layer("full_down_T57600", 57600, 13824, 5120, 0.7, 64, 0, X_DOWN, W_
 
 
 def sweep_layers():
-    """The 16-point sweep at T=16384 on the up-projection shape."""
+    """The sweep at T=16384 on the up-projection shape: k x weight-scale layout
+    (32x1, 32x32, 128x1) x alpha."""
     out = []
     for k in (0, 16, 64, 256):
-        for layout in (0, 1):
+        for layout in (0, 1, 2):
             for alpha in (0.5, 0.7):
                 out.append(Layer(f"sweep_k{k}_l{layout}_a{alpha}", 16384, 5120, 13824,
                                  alpha, k, layout, X_UP, W_UP))

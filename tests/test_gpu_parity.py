@@ -25,6 +25,7 @@ TINY = synth.TINY
 RAGGED = synth.Layer("ragged", 200, 136, 368, 0.6, 3, 0, synth.XSpec("student3", 0.3, 4, 8.0, 30.0),
                      synth.WSpec(0.02))
 RAGGED32 = RAGGED.with_(name="ragged_32x32", layout=1, k=11)
+RAGGED128 = RAGGED.with_(name="ragged_128x1", layout=2, k=7, d_in=904)   # partial last stripe
 K0 = TINY.with_(name="k0", k=0)
 KFULL = synth.Layer("kfull", 300, 64, 272, 0.5, 64, 0, synth.X_TINY, synth.WSpec(0.02))
 T1 = TINY.with_(name="T1", T=1)
@@ -34,7 +35,9 @@ FFN2 = synth.FFN2
 
 SINGLE = RAGGED.with_(name="ragged_T100_single_cta", T=100, k=5)   # T <= 128: single-CTA GEMM
 
-SMALL = [TINY, RAGGED, RAGGED32, K0, KFULL, T1, SINGLE]
+MID128 = MID.with_(name="mid_k64_128x1", layout=2, k=64)
+
+SMALL = [TINY, RAGGED, RAGGED32, RAGGED128, K0, KFULL, T1, SINGLE]
 
 
 def _calibrate(L):
@@ -152,7 +155,7 @@ def test_topk_ties_go_to_lower_index():
 # ---------------------------------------------------------------------------
 # Weight packing
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("L", SMALL + [MID, FFN0], ids=lambda L: L.name)
+@pytest.mark.parametrize("L", SMALL + [MID, MID128, FFN0], ids=lambda L: L.name)
 def test_pack_parity(L):
     X, W, pw = _calibrate(L)
     c = gu.oracle_calib_from_gpu(pw)
@@ -165,7 +168,14 @@ def test_pack_parity(L):
     if d.nblk:
         sfb = gu.sf_canonical(pw.sfb, d.sfb_rows, d.nblk, nb_ref)
         np.testing.assert_array_equal(sfb[:L.d_out, :nb_ref], ref["sfb"])
-        assert not sfb[L.d_out:].any() and not sfb[:, nb_ref:].any()
+        assert not sfb[L.d_out:].any()
+        tail = nb_ref
+        if L.layout == w4.SF_128x1_KMAJOR:
+            # padding blocks inside the last, partial stripe carry its code
+            tail = -(-nb_ref // 4) * 4
+            for b in range(nb_ref, tail):
+                np.testing.assert_array_equal(sfb[:L.d_out, b], sfb[:L.d_out, nb_ref - 1])
+        assert not sfb[:, tail:].any()
     w_hp = gu.bf16_bits(pw.w_hp).reshape(L.d_out, d.k_pad)
     np.testing.assert_array_equal(w_hp[:, :L.k], ref["w_hp"])
     assert not w_hp[:, L.k:].any()
@@ -213,7 +223,7 @@ def _linear(X, pw, T, d_out):
     return Y
 
 
-@pytest.mark.parametrize("L", SMALL + [MID], ids=lambda L: L.name)
+@pytest.mark.parametrize("L", SMALL + [MID, MID128], ids=lambda L: L.name)
 def test_linear_parity_full_output(L):
     X, W, pw = _calibrate(L)
     Y = _linear(X, pw, L.T, L.d_out)

@@ -26,7 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(6)
 NOALLOC_SCRATCH_BYTES = 32 << 20     # W4A4_NOALLOC_SCRATCH_BYTES
-SF_32x1_KMAJOR, SF_32x32_TILE = 0, 1
+SF_32x1_KMAJOR, SF_32x32_TILE, SF_128x1_KMAJOR = 0, 1, 2
 
 _i64 = ctypes.c_int64
 _vp = ctypes.c_void_p

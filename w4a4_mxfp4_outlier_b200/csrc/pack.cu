@@ -83,16 +83,18 @@ __global__ void pack_o_kernel(const uint16_t* __restrict__ W, int64_t ldw,
 cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,
                         const int32_t* jmap, const Geometry& g, int layout, uint8_t* wq,
                         uint8_t* sfb, void* w_hp, cudaStream_t stream) {
-  if (layout == 0) {
-    // 32x1 stripes: the fold w * s_j, the compaction, the per-row 1x32 block
-    // encoding and the bf16 outlier columns are exactly what the activation
-    // prep computes with s in place of inv_s, so the rows of W stream through
-    // the prep kernel (scale rows d_out .. sfb_rows are zeroed first).
+  if (layout == W4A4_SF_32x1_KMAJOR || layout == W4A4_SF_128x1_KMAJOR) {
+    // 32x1 / 128x1 stripes: the fold w * s_j, the compaction, the per-row
+    // block encoding and the bf16 outlier columns are exactly what the
+    // activation prep computes with s in place of inv_s (128x1: the amax
+    // reduced over 4 blocks), so the rows of W stream through the prep
+    // kernel (scale rows d_out .. sfb_rows are zeroed first).
     if (g.nblk > 0) {
       cudaError_t e = cudaMemsetAsync(sfb, 0, static_cast<size_t>(g.sfb_rows * g.nblk), stream);
       if (e != cudaSuccess) return e;
     }
-    return launch_prep(W, g.d_out, ldw, s, O, jmap, g, wq, sfb, w_hp, stream);
+    return launch_prep(W, g.d_out, ldw, s, O, jmap, g, wq, sfb, w_hp, stream,
+                       layout == W4A4_SF_128x1_KMAJOR);
   }
   if (g.nblk > 0) {
     const int64_t warps = (g.sfb_rows / 32) * g.nblk;

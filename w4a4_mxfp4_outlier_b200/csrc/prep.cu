@@ -50,7 +50,8 @@ template <int CH>
 __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t ldx, int d_in,
                 const float* __restrict__ inv_s, const int32_t* __restrict__ O,
                 const int32_t* __restrict__ jmap, int k, int k_pad, int kj, int nchunks, int nblk,
-                uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa, uint32_t* __restrict__ xo) {
+                uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa, uint32_t* __restrict__ xo,
+                int stripe4) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kPrepStages) * kPrepStage);
   uint64_t* empty = full + kPrepStages;
@@ -190,6 +191,10 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
           }
           amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
           amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+          if (stripe4) {                      // 128x1 stripes: 16 lanes, 4 blocks
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 8));
+          }
           const uint32_t code = mx_scale_code(amax);
           const float inv = mx_inv_scale(code);
           const float2 inv2 = make_float2(inv, inv);
@@ -265,7 +270,7 @@ template <int CH>
 static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, int64_t T,
                                   int64_t ldx, const float* inv_s, const int32_t* O,
                                   const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                                  uint8_t* sfa, void* xo, cudaStream_t stream) {
+                                  uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4) {
   cudaError_t e = cudaFuncSetAttribute(prep_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kPrepSmem));
   if (e != cudaSuccess) return e;
@@ -273,21 +278,21 @@ static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, in
       static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
       static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
       static_cast<int>(g.kj_pad / 8), static_cast<int>(g.nblk), aq, sfa,
-      static_cast<uint32_t*>(xo));
+      static_cast<uint32_t*>(xo), stripe4 ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
                         const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                        uint8_t* sfa, void* xo, cudaStream_t stream) {
+                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4) {
   if (T == 0) return cudaSuccess;
   const PrepPlan p = plan_prep(g);
   const int sms = device_num_sms();
   const int grid = static_cast<int>(T < sms ? T : sms);
   switch (p.ch) {
-    case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
-    case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
-    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream);
+    case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
+    case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
+    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
   }
 }
 

@@ -30,7 +30,8 @@ static w4a4_status check_pw(const w4a4_packed_weight* pw, Geometry* g) {
   if (pw == nullptr) return W4A4_ERR_INVALID_ARG;
   w4a4_status st = check_dims(pw->d_in, pw->d_out, pw->k);
   if (st != W4A4_OK) return st;
-  if (pw->layout != W4A4_SF_32x1_KMAJOR && pw->layout != W4A4_SF_32x32_TILE)
+  if (pw->layout != W4A4_SF_32x1_KMAJOR && pw->layout != W4A4_SF_32x32_TILE &&
+      pw->layout != W4A4_SF_128x1_KMAJOR)
     return W4A4_ERR_INVALID_ARG;
   *g = make_geometry(pw->d_in, pw->d_out, pw->k);
   if (g->kj > 0 && (pw->wq == nullptr || pw->sfb == nullptr || pw->jmap == nullptr))

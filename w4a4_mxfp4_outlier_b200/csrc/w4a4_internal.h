@@ -52,9 +52,10 @@ int finalize_max_d();
 cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,
                         const int32_t* jmap, const Geometry& g, int layout, uint8_t* wq,
                         uint8_t* sfb, void* w_hp, cudaStream_t stream);
+// stripe4 = true: one exponent per 4 consecutive blocks (128x1 weight stripes)
 cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
                         const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                        uint8_t* sfa, void* xo, cudaStream_t stream);
+                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4 = false);
 bool prep_supported(const Geometry& g);
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
                         const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,

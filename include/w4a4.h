@@ -48,7 +48,8 @@ typedef enum w4a4_status {
   W4A4_ERR_UNSUPPORTED_SHAPE = 2,/* alignment or size outside the supported set above */
   W4A4_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
   W4A4_ERR_TIMEOUT = 4,          /* a device pipeline wait ran out (see w4a4_last_error) */
-  W4A4_ERR_SCRATCH_LIMIT = 5     /* the problem needs more scratch than w4a4_linear_noalloc has */
+  W4A4_ERR_SCRATCH_LIMIT = 5,    /* the problem needs more scratch than w4a4_linear_noalloc has */
+  W4A4_ERR_BAD_IMAGE = 6         /* a packed-weight image failed its magic, version, size or checksum check */
 } w4a4_status;
 
 /* Weight scale layouts of the block packing (review sec. 3.4: "32x32 tiles"
@@ -197,6 +198,40 @@ w4a4_status w4a4_linear(const void* X, int64_t T, int64_t ldx, const w4a4_packed
 w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_weight* pw,
                              void* X_dev, void* workspace, size_t ws_bytes, void* Y_dev,
                              void* Y_host, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packed-weight images (checkpoints).  The offline result of a layer --
+ * Wq, SFB, W_hp, s, inv_s, O, jmap -- as one host byte image: a 256-byte
+ * header (magic "W4A4PKW1", format version, layout, d_in, d_out, k, the
+ * section sizes, an FNV-1a 64 checksum of the section bytes) followed by the
+ * sections in that order, each padded to 64 bytes.  The review's static O and
+ * offline fold (sec. 3.3, 3.5) make this record the complete state of a
+ * quantised layer.  Host buffers are caller-owned; pinned memory makes the
+ * copies faster.  Each call synchronises `stream`.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of the image of *pw. */
+w4a4_status w4a4_packed_image_size(const w4a4_packed_weight* pw, size_t* bytes);
+
+/* Writes the image of *pw (device buffers named in the record, plus s, a
+ * float32 [d_in] device array) to host[0 .. bytes).  INVALID_ARG if bytes is
+ * below w4a4_packed_image_size or a needed pointer is NULL. */
+w4a4_status w4a4_packed_save(const w4a4_packed_weight* pw, const float* s, void* host,
+                             size_t bytes, void* stream);
+
+/* Reads the header of an image: d_in, d_out, k, layout (any output pointer
+ * may be NULL), so a caller can allocate the buffers before loading.
+ * BAD_IMAGE on a wrong magic or version, inconsistent sizes, a short buffer
+ * or a checksum mismatch. */
+w4a4_status w4a4_packed_image_info(const void* host, size_t bytes, int64_t* d_in, int64_t* d_out,
+                                   int64_t* k, int32_t* layout);
+
+/* Copies an image into the device buffers the record *pw names (its inv_s,
+ * O and jmap arrays are written too) and into s.  The record's d_in, d_out,
+ * k and layout must equal the image's (else INVALID_ARG); BAD_IMAGE as for
+ * w4a4_packed_image_info. */
+w4a4_status w4a4_packed_load(const void* host, size_t bytes, const w4a4_packed_weight* pw,
+                             float* s, void* stream);
 
 /* Size of the fixed device scratch array behind w4a4_linear_noalloc. */
 #define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -133,3 +133,24 @@ def test_prep_width_limit():
     assert w4._prep_act(0x1000, 8, 16392, ctypes.byref(pw), 0x1000, 0x1000, 0x1000, None) \
         == w4.ERR_UNSUPPORTED_SHAPE
 
+
+def test_packed_image_header_checks():
+    # no GPU needed: the header is checked before anything is copied
+    import numpy as np
+    img = np.zeros(4096, np.uint8)
+    d = ctypes.c_int64()
+    st = w4._packed_image_info(img.ctypes.data, img.size, ctypes.byref(d), None, None, None)
+    assert st == w4.ERR_BAD_IMAGE                       # no magic
+    assert w4._packed_image_info(None, 0, None, None, None, None) == w4.ERR_BAD_IMAGE
+    img[:8] = np.frombuffer(b"W4A4PKW1", np.uint8)
+    assert w4._packed_image_info(img.ctypes.data, img.size, None, None, None, None) \
+        == w4.ERR_BAD_IMAGE                             # version 0, zero sizes
+    assert "checksum" in w4.status_string(w4.ERR_BAD_IMAGE)
+    pw = _raw_pw()
+    n = ctypes.c_size_t()
+    assert w4._packed_image_size(ctypes.byref(pw), ctypes.byref(n)) == w4.OK
+    # header slot + sections, each padded to 64 bytes
+    d = w4.get_dims(64, 32, 4)
+    sizes = [32 * d.kj_pad // 2, d.sfb_rows * d.nblk, 32 * d.k_pad * 2, 256, 256, 16, 240]
+    assert n.value == 256 + sum(-(-x // 64) * 64 for x in sizes)
+

@@ -24,7 +24,8 @@ if not os.path.exists(LIB_PATH):
                       "`python w4a4_mxfp4_outlier_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(6)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT,
+ ERR_BAD_IMAGE) = range(7)
 NOALLOC_SCRATCH_BYTES = 32 << 20     # W4A4_NOALLOC_SCRATCH_BYTES
 SF_32x1_KMAJOR, SF_32x32_TILE, SF_128x1_KMAJOR = 0, 1, 2
 
@@ -75,6 +76,15 @@ _linear_host = _sig("w4a4_linear_host", _st, _vp, _i64, ctypes.POINTER(PackedWei
                     ctypes.c_size_t, _vp, _vp, _vp)
 _linear_noalloc = _sig("w4a4_linear_noalloc", _st, _vp, _i64, _i64, ctypes.POINTER(PackedWeightC),
                        _vp, _i64, _vp)
+_packed_image_size = _sig("w4a4_packed_image_size", _st, ctypes.POINTER(PackedWeightC),
+                          ctypes.POINTER(ctypes.c_size_t))
+_packed_save = _sig("w4a4_packed_save", _st, ctypes.POINTER(PackedWeightC), _vp, _vp,
+                    ctypes.c_size_t, _vp)
+_packed_image_info = _sig("w4a4_packed_image_info", _st, _vp, ctypes.c_size_t,
+                          ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64),
+                          ctypes.POINTER(ctypes.c_int32))
+_packed_load = _sig("w4a4_packed_load", _st, _vp, ctypes.c_size_t, ctypes.POINTER(PackedWeightC),
+                    _vp, _vp)
 _last_error = _sig("w4a4_last_error", _st, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32))
 
 EXPORTED = [
@@ -82,6 +92,7 @@ EXPORTED = [
     "w4a4_calib_observe", "w4a4_calib_finalize", "w4a4_weight_sizes", "w4a4_pack_weight",
     "w4a4_workspace_size", "w4a4_prep_act", "w4a4_gemm_dual", "w4a4_linear",
     "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
+    "w4a4_packed_image_size", "w4a4_packed_save", "w4a4_packed_image_info", "w4a4_packed_load",
 ]
 
 
@@ -274,6 +285,43 @@ def linear_noalloc(X: torch.Tensor, pw: PackedWeight, Y: torch.Tensor, stream=No
     c = pw.c
     _check(_linear_noalloc(_ptr(X), X.shape[0], X.stride(0), ctypes.byref(c), _ptr(Y), Y.stride(0),
                            _stream(stream)), "linear_noalloc")
+
+
+def packed_to_bytes(pw: PackedWeight, stream=None) -> bytes:
+    """The checkpoint image of a packed layer (see w4a4_packed_save)."""
+    c = pw.c
+    n = ctypes.c_size_t()
+    _check(_packed_image_size(ctypes.byref(c), ctypes.byref(n)), "packed_image_size")
+    buf = torch.empty(n.value, dtype=torch.uint8, pin_memory=torch.cuda.is_available())
+    _check(_packed_save(ctypes.byref(c), _ptr(pw.s), buf.data_ptr(), n.value, _stream(stream)),
+           "packed_save")
+    return buf.numpy().tobytes()
+
+
+def packed_from_bytes(image: bytes, device="cuda", stream=None) -> PackedWeight:
+    """Allocates a packed layer on `device` and loads a checkpoint image into
+    it.  act_scale, w_scale and score are not part of the image (zeros)."""
+    buf = torch.frombuffer(bytearray(image), dtype=torch.uint8)
+    d_in, d_out, k, layout = _i64(), _i64(), _i64(), ctypes.c_int32()
+    _check(_packed_image_info(buf.data_ptr(), buf.numel(), ctypes.byref(d_in), ctypes.byref(d_out),
+                              ctypes.byref(k), ctypes.byref(layout)), "packed_image_info")
+    pw = alloc_packed(d_in.value, d_out.value, k.value, layout.value, device)
+    for t in (pw.act_scale, pw.w_scale, pw.score):
+        t.zero_()
+    c = pw.c
+    _check(_packed_load(buf.data_ptr(), buf.numel(), ctypes.byref(c), _ptr(pw.s), _stream(stream)),
+           "packed_load")
+    return pw
+
+
+def save_packed(pw: PackedWeight, path: str, stream=None):
+    with open(path, "wb") as f:
+        f.write(packed_to_bytes(pw, stream))
+
+
+def load_packed(path: str, device="cuda", stream=None) -> PackedWeight:
+    with open(path, "rb") as f:
+        return packed_from_bytes(f.read(), device, stream)
 
 
 def last_error(clear: bool = True, stream=None):

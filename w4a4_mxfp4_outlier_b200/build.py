@@ -24,7 +24,8 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["libw4a4.cu"]
 HEADERS = ["w4a4_device.cuh", "w4a4_internal.h", "w4a4_api.cu", "calib.cu", "prep.cu",
-           "pack.cu", "gemm.cu", "noalloc.cu"]
+           "pack.cu", "gemm.cu", "noalloc.cu",
+           "checkpoint.cu"]
 
 
 def nvcc() -> str:

@@ -7,3 +7,4 @@
 #include "prep.cu"
 #include "gemm.cu"
 #include "noalloc.cu"
+#include "checkpoint.cu"

@@ -77,6 +77,7 @@ const char* w4a4_status_string(w4a4_status s) {
     case W4A4_ERR_CUDA: return "CUDA error";
     case W4A4_ERR_TIMEOUT: return "device pipeline wait timed out";
     case W4A4_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed no-alloc scratch";
+    case W4A4_ERR_BAD_IMAGE: return "packed-weight image failed its header or checksum check";
   }
   return "unknown status";
 }

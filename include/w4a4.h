@@ -263,6 +263,15 @@ w4a4_status w4a4_linear_noalloc(const void* X, int64_t T, int64_t ldx,
                                 const w4a4_packed_weight* pw, void* Y, int64_t ldy,
                                 void* stream);
 
+/* Layer-wise parameter choice (review sec. 4 table and sec. 6: alpha and k
+ * per layer are the next step; the pages give no procedure).  Sums over a
+ * T x d_out block, in float64: sums[0] = sum (Y - Yref)^2, sums[1] =
+ * sum Yref^2, with Y bf16 (row stride ldy) and Yref float32 (row stride ldr);
+ * sums is a device array of 2 doubles, zeroed by the call.  A search scores a
+ * candidate (alpha, k, layout) by sqrt(sums[0] / sums[1]). */
+w4a4_status w4a4_error_sums(const void* Y, int64_t ldy, const float* Yref, int64_t ldr, int64_t T,
+                            int64_t d_out, double* sums, void* stream);
+
 /* Synchronises `stream` and reports device-side failures recorded since the
  * last clear: W4A4_OK, or W4A4_ERR_TIMEOUT if a bounded wait ran out (the
  * affected output is incomplete).  *bits (may be NULL) receives the raw

@@ -378,6 +378,31 @@ def linear_reference(X: np.ndarray, W: np.ndarray, alpha: float, k: int,
     return Y, {**c, **pw, **pa}
 
 
+def search_layer(X: np.ndarray, W: np.ndarray, alphas, ks, layouts=(LAYOUT_32x1,), X_eval=None):
+    """Layer-wise (alpha, k, layout) choice [review sec. 4 table "Layer-wise
+    alpha and k"; sec. 6 "next step"; no procedure given]: for every
+    candidate the quantised layer's Y on X_eval (default X, calibration on X)
+    is compared with the exact float64 product X_eval W^T; the smallest
+    relative Frobenius error wins, the smaller k on ties.
+    Returns (best, {candidate: error})."""
+    Xe = X if X_eval is None else X_eval
+    exact = Xe.astype(np.float64) @ W.astype(np.float64).T
+    den = float(np.sum(exact * exact))
+    errors = {}
+    for layout in layouts:
+        for k in ks:
+            for alpha in alphas:
+                c = calibrate(X, W, alpha, k)
+                pw = pack_weight(W, c["s"], c["O"], c["J"], layout)
+                pa = prep_activation(Xe, c["inv_s"], c["O"], c["J"])
+                Y = dual_branch_product(pa["aq"], pa["sfa"], pa["xo"], pw["wq"], pw["sfb"],
+                                        pw["w_hp"])
+                errors[(alpha, k, layout)] = float(np.sqrt(np.sum((Y - exact) ** 2) / den)) \
+                    if den > 0 else 0.0
+    best = min(errors, key=lambda cnd: (errors[cnd], cnd[1]))
+    return best, errors
+
+
 def mma_sf_offset(r, kb, nblk: int):
     """Byte offset of scale (row r, block kb) in the block-scaled MMA layout.
 

@@ -277,6 +277,21 @@ def test_128x1_stripes_share_scale_and_saturate_at_max():
                 assert codes[r, i] in (6, 7)
 
 
+def test_search_layer_prefers_protecting_planted_outliers():
+    """On the tiny workload (8 planted heavy channels), keeping them in bf16
+    (k = 8) beats k = 0 at every alpha, all-bf16 (k = d_in) is near exact,
+    and the returned best is the table's minimum."""
+    L = synth.TINY
+    Xt, Wt = synth.gen_layer(L, "cpu")
+    X, W = Xt.float().numpy()[:64], Wt.float().numpy()
+    best, err = orc.search_layer(X, W, alphas=(0.3, 0.5, 0.7), ks=(0, 8, L.d_in))
+    for a in (0.3, 0.5, 0.7):
+        assert err[(a, 8, 0)] < 0.8 * err[(a, 0, 0)]
+        assert err[(a, L.d_in, 0)] < 5e-3          # bf16 rounding of smoothed operands only
+    assert best == min(err, key=lambda c: (err[c], c[1]))
+    assert best[1] == L.d_in
+
+
 def test_tiny_generator_matches_pages_statistics():
     """The tiny workload's planted channels exceed 6.0, weights stay below 0.6
     (review §3.1), and after smoothing the planted channels are the top-8."""

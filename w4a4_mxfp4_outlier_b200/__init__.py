@@ -85,6 +85,7 @@ _packed_image_info = _sig("w4a4_packed_image_info", _st, _vp, ctypes.c_size_t,
                           ctypes.POINTER(ctypes.c_int32))
 _packed_load = _sig("w4a4_packed_load", _st, _vp, ctypes.c_size_t, ctypes.POINTER(PackedWeightC),
                     _vp, _vp)
+_error_sums = _sig("w4a4_error_sums", _st, _vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp)
 _last_error = _sig("w4a4_last_error", _st, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32))
 
 EXPORTED = [
@@ -93,6 +94,7 @@ EXPORTED = [
     "w4a4_workspace_size", "w4a4_prep_act", "w4a4_gemm_dual", "w4a4_linear",
     "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
     "w4a4_packed_image_size", "w4a4_packed_save", "w4a4_packed_image_info", "w4a4_packed_load",
+    "w4a4_error_sums",
 ]
 
 

@@ -8,3 +8,4 @@
 #include "gemm.cu"
 #include "noalloc.cu"
 #include "checkpoint.cu"
+#include "metrics.cu"

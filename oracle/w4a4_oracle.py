@@ -84,6 +84,61 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# FFN activation between the two projections
+# ----------------------------------------------------------------------------
+# The review quantises both FFN projections of the Wan2.2 DiT (ffn.0 and
+# ffn.2, §3.1/§3.5); between them the FFN applies GELU (tanh form), which the
+# pages do not write out.  The fused up->down step feeds the down projection
+# with X_down = bf16_rn(gelu(bf16 Y_up)).  Because the GELU value decides
+# quantised codes, the oracle takes that decision in the kernel's precision,
+# float32, with one fixed sequence of IEEE operations (every product, sum and
+# quotient separately rounded, no fused multiply-add):
+#
+#   gelu(x) = x / (1 + exp(z)),  z = clamp(-2 * 0.7978845608 * (x + 0.044715 x^3), -87, 88)
+#
+# (0.5 x (1 + tanh(u)) = x / (1 + exp(-2u))), with exp by Cody-Waite range
+# reduction z = n ln2 + r (n = round-half-even(z log2 e), ln2 split into a
+# high part exact in 16 bits and a low part) and the degree-7 Taylor
+# polynomial of exp(r) on |r| <= 0.35 in Horner form, times 2^n.
+
+_F = np.float32
+_LOG2E = _F(1.4426950408889634)
+_LN2_HI = _F(0.693145751953125)          # 0x3F317200: 16 significant bits, n * LN2_HI exact
+_LN2_LO = _F(1.428606765330187e-06)      # ln 2 - LN2_HI
+_EXP_C = [_F(1.0 / 5040), _F(1.0 / 720), _F(1.0 / 120), _F(1.0 / 24), _F(1.0 / 6), _F(0.5),
+          _F(1.0), _F(1.0)]               # Horner order, highest degree first
+_GELU_A = _F(-2.0 * 0.7978845608028654)  # -2 sqrt(2 / pi)
+_GELU_B = _F(0.044715)
+
+
+def exp_f32(z: np.ndarray) -> np.ndarray:
+    """exp of float32 z in [-87, 88] by the steps above (float32 arithmetic)."""
+    z = np.asarray(z, dtype=np.float32)
+    n = np.rint(z * _LOG2E).astype(np.float32)                   # ties to even
+    r = (z - n * _LN2_HI) - n * _LN2_LO
+    p = np.full_like(r, _EXP_C[0])
+    for c in _EXP_C[1:]:
+        p = p * r + c
+    scale = ((n.astype(np.int32) + 127).astype(np.uint32) << 23).view(np.float32)
+    return (p * scale).astype(np.float32)
+
+
+def gelu_f32(x: np.ndarray) -> np.ndarray:
+    """GELU (tanh form) of float32 x, as defined above."""
+    x = np.asarray(x, dtype=np.float32)
+    x3 = (x * x) * x
+    z = _GELU_A * (x + _GELU_B * x3)
+    z = np.minimum(np.maximum(z, _F(-87.0)), _F(88.0))
+    with np.errstate(over="ignore", invalid="ignore"):
+        return (x / (_F(1.0) + exp_f32(z))).astype(np.float32)
+
+
+def ffn_hidden(Y_up: np.ndarray) -> np.ndarray:
+    """X_down = bf16_rn(gelu(Y_up)) for bf16-exact float32 Y_up."""
+    return bf16_bits_to_f32(f32_to_bf16_bits(gelu_f32(Y_up)))
+
+
+# ----------------------------------------------------------------------------
 # Calibration  [review §3.2 "collect per-channel magnitudes"; §3.1]
 # ----------------------------------------------------------------------------
 

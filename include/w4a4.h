@@ -233,6 +233,51 @@ w4a4_status w4a4_packed_image_info(const void* host, size_t bytes, int64_t* d_in
 w4a4_status w4a4_packed_load(const void* host, size_t bytes, const w4a4_packed_weight* pw,
                              float* s, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The FFN pair (review sec. 3.1, 3.5: both FFN projections, ffn.0 up and
+ * ffn.2 down, take the same W4A4 recipe).  Between them the Wan2.2 FFN
+ * applies GELU, which the pages do not write out; here X_down =
+ * bf16_rn(gelu(bf16 Y_up)) with GELU in tanh form evaluated in float32 by a
+ * fixed sequence of IEEE operations: gelu(x) = x / (1 + exp(z)), z =
+ * clamp(-2 sqrt(2/pi) (x + 0.044715 x^3), -87, 88), exp by Cody-Waite
+ * reduction and a degree-7 Taylor polynomial (|error| < 1e-6 against the
+ * exact tanh form).
+ *
+ * Fused use: calibrate and pack the down layer, w4a4_ffn_link it, pack the up
+ * weight with w4a4_pack_weight_rows(rows = perm), then per batch
+ * w4a4_prep_act (up) -> w4a4_gemm_dual_act (up, writing the down layer's Aq,
+ * SFA, X_O) -> w4a4_gemm_dual (down).
+ * ------------------------------------------------------------------------ */
+
+/* X[t, j] = bf16_rn(gelu(Y[t, j])) for a bf16 [T, d] matrix (row strides
+ * ldy, ldx elements); the unfused activation, e.g. to calibrate the down
+ * layer. */
+w4a4_status w4a4_gelu_bf16(const void* Y, int64_t T, int64_t d, int64_t ldy, void* X, int64_t ldx,
+                           void* stream);
+
+/* For a packed down layer `next`: perm[c] (int32 [d_in]) = jmap[c] for
+ * c < kj, O[c - kj] after, and inv_s_perm[c] = inv_s[perm[c]] (float32
+ * [d_in]): the up layer's output-channel order under which the down layer's
+ * compacted input is contiguous. */
+w4a4_status w4a4_ffn_link(const w4a4_packed_weight* next, int32_t* perm, float* inv_s_perm,
+                          void* stream);
+
+/* w4a4_pack_weight with the rows of W permuted: packed output channel n is
+ * W row rows[n] (rows: int32 [d_out] device array). */
+w4a4_status w4a4_pack_weight_rows(const void* W, int64_t ldw, const float* s, const int32_t* rows,
+                                  const w4a4_packed_weight* pw, void* stream);
+
+/* The up projection with the fused FFN epilogue: computes the dual-branch
+ * product of (aq, sfa, xo) with pw (packed with rows = perm) and, instead of
+ * storing Y, writes the down layer's activation buffers as w4a4_prep_act
+ * would for X = bf16_rn(gelu(bf16 Y)) in its original channel order:
+ * aq_next [T, kj_pad/2], sfa_next (MMA layout), xo_next bf16 [T, k_pad].
+ * next->d_in must equal pw->d_out.  inv_s_perm from w4a4_ffn_link. */
+w4a4_status w4a4_gemm_dual_act(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                               const w4a4_packed_weight* pw, const w4a4_packed_weight* next,
+                               const float* inv_s_perm, uint8_t* aq_next, uint8_t* sfa_next,
+                               void* xo_next, void* stream);
+
 /* Size of the fixed device scratch array behind w4a4_linear_noalloc. */
 #define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 

@@ -126,10 +126,10 @@ def exp_f32(z: np.ndarray) -> np.ndarray:
 def gelu_f32(x: np.ndarray) -> np.ndarray:
     """GELU (tanh form) of float32 x, as defined above."""
     x = np.asarray(x, dtype=np.float32)
-    x3 = (x * x) * x
-    z = _GELU_A * (x + _GELU_B * x3)
-    z = np.minimum(np.maximum(z, _F(-87.0)), _F(88.0))
-    with np.errstate(over="ignore", invalid="ignore"):
+    with np.errstate(over="ignore", invalid="ignore"):      # |x|^3 may overflow to inf
+        x3 = (x * x) * x
+        z = _GELU_A * (x + _GELU_B * x3)
+        z = np.minimum(np.maximum(z, _F(-87.0)), _F(88.0))
         return (x / (_F(1.0) + exp_f32(z))).astype(np.float32)
 
 

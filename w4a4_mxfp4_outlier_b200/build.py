@@ -25,7 +25,7 @@ LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["libw4a4.cu"]
 HEADERS = ["w4a4_device.cuh", "w4a4_internal.h", "w4a4_api.cu", "calib.cu", "prep.cu",
            "pack.cu", "gemm.cu", "noalloc.cu",
-           "checkpoint.cu", "metrics.cu"]
+           "checkpoint.cu", "metrics.cu", "ffn.cu"]
 
 
 def nvcc() -> str:

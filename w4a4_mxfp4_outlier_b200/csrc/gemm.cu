@@ -76,7 +76,63 @@ struct GemmArgs {
   int kt_j;          // MXFP4 K tiles (256 columns each)
   int k_pad;         // bf16 columns (multiple of 16)
   int tiles_m, tiles_n;
+  // Fused FFN epilogue (kernels instantiated with kAct): Y is not stored;
+  // column c of the tile row feeds the next layer, whose input channel c is
+  // its compacted J position c for c < act_kj and outlier c - act_kj after:
+  //   v = fl32(bf16(gelu(bf16(acc))) * act_inv_s[c])
+  // J blocks are MXFP4-encoded into act_aq / act_sfa, outliers go to act_xo.
+  const float* act_inv_s;   // [d_out] inv_s of the next layer in this column order
+  uint8_t* act_aq;          // [T, act_nblk * 16]
+  uint8_t* act_sfa;         // MMA layout, act_nblk blocks per row
+  __nv_bfloat16* act_xo;    // [T, act_k_pad]
+  int act_kj, act_nblk, act_k_pad;
 };
+
+// One lane's 32 accumulator columns col0 .. col0+31 of row `row` through the
+// fused FFN epilogue (see GemmArgs).  No warp collectives: callable per lane.
+__device__ __forceinline__ void act_block(const uint32_t (&acc)[32], int row, int col0,
+                                          const GemmArgs& a) {
+  if (row >= a.T) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int col = col0 + i;
+    const float y = __bfloat162float(__float2bfloat16_rn(__uint_as_float(acc[i])));
+    const float x = __bfloat162float(__float2bfloat16_rn(ffn_gelu(y)));
+    v[i] = col < a.d_out ? __fmul_rn(x, a.act_inv_s[col]) : 0.0f;
+  }
+  // outlier columns of the next layer (and its zero padding up to k_pad)
+  if (col0 + 32 > a.act_kj && col0 < a.act_kj + a.act_k_pad) {
+    __nv_bfloat16* xr = a.act_xo + static_cast<int64_t>(row) * a.act_k_pad;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int o = col0 + i - a.act_kj;
+      if (o >= 0 && o < a.act_k_pad) xr[o] = __float2bfloat16_rn(v[i]);
+    }
+  }
+  // the MX block of compacted positions col0 .. col0+31 (zeros past act_kj)
+  const int b = col0 >> 5;
+  if (b < a.act_nblk) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (col0 + i >= a.act_kj) v[i] = 0.0f;
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+    const uint32_t code = mx_scale_code(amax);
+    const float inv = mx_inv_scale(code);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q], inv), __fmul_rn(v[8 * q + 1], inv),
+                        __fmul_rn(v[8 * q + 2], inv), __fmul_rn(v[8 * q + 3], inv),
+                        __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
+                        __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
+    *reinterpret_cast<uint4*>(a.act_aq + static_cast<int64_t>(row) * a.act_nblk * 16 + b * 16) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+    a.act_sfa[sf_offset(row, b, a.act_nblk)] = static_cast<uint8_t>(code);
+  }
+}
 
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
   const int per_group = GROUP_M * tiles_n;
@@ -88,6 +144,7 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   tm = first_m + w % gm;
 }
 
+template <bool kAct>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
@@ -276,7 +333,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (lane == 0) mbar_arrive(&sm.acc_empty);
 
       const int row = tm * BM + 32 * sp + lane;
-      if (row < args.T) {
+      if constexpr (kAct) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) act_block(r[c], row, tn * BN + 128 * half + 32 * c, args);
+      } else if (row < args.T) {
         __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -346,6 +406,7 @@ struct PairSmem {
   uint32_t abort_flag;
 };
 
+template <bool kAct>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
@@ -579,6 +640,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
+      if constexpr (kAct) {
+        const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) act_block(r[c], row, tn * 256 + 128 * half + 32 * c, args);
+        continue;
+      }
       // Y through a per-warp staging block, 16 rows x 32 columns at a time:
       // the lanes holding those rows write them (64-byte swizzle: 16-byte
       // chunk j of row r sits at chunk j ^ ((r >> 1) & 3), so the writes hit
@@ -685,7 +752,9 @@ static int pair_capacity() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] > 0) return cached[dev];
   const size_t smem = gemm_pair_smem_bytes();
-  if (cudaFuncSetAttribute(gemm_dual_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(gemm_dual_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(gemm_dual_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
@@ -700,8 +769,12 @@ static int pair_capacity() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel, &cfg) != cudaSuccess || n <= 0)
+  int n2 = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel<false>, &cfg) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n2, gemm_dual_pair_kernel<true>, &cfg) != cudaSuccess ||
+      n <= 0 || n2 <= 0)
     return 0;
+  if (n2 < n) n = n2;
   cached[dev] = n;
   return n;
 }
@@ -712,7 +785,7 @@ constexpr int64_t kPairMinT = 129;
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
                         const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
-                        void* Y, int64_t ldy, cudaStream_t stream) {
+                        void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act) {
   if (T == 0 || g.d_out == 0) return cudaSuccess;
   const bool pair = T >= kPairMinT && pair_capacity() > 0;
   const uint32_t brows = pair ? 128 : BN;
@@ -758,6 +831,13 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   a.k_pad = static_cast<int>(g.k_pad);
   a.tiles_m = static_cast<int>((T + (pair ? 255 : BM - 1)) / (pair ? 256 : BM));
   a.tiles_n = static_cast<int>((g.d_out + BN - 1) / BN);
+  a.act_inv_s = act ? act->inv_s : nullptr;
+  a.act_aq = act ? act->aq : nullptr;
+  a.act_sfa = act ? act->sfa : nullptr;
+  a.act_xo = act ? static_cast<__nv_bfloat16*>(act->xo) : nullptr;
+  a.act_kj = act ? static_cast<int>(act->kj) : 0;
+  a.act_nblk = act ? static_cast<int>(act->nblk) : 0;
+  a.act_k_pad = act ? static_cast<int>(act->k_pad) : 0;
   const int ntiles = a.tiles_m * a.tiles_n;
   if (pair) {
     const int npairs = ntiles < pair_capacity() ? ntiles : pair_capacity();
@@ -777,19 +857,31 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
     // Y as bf16 tiles of 16 rows x 32 columns, 64-byte swizzle (epilogue staging layout)
     CUtensorMap tm_y;
     memset(&tm_y, 0, sizeof(tm_y));
+    if (act != nullptr)
+      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true>, tm_a, tm_b, tm_ao, tm_bo,
+                                tm_sfa, tm_sfb, tm_y, a);
     if (!make_tmap(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
                    static_cast<uint64_t>(ldy) * 2, 16, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel, tm_a, tm_b, tm_ao, tm_bo, tm_sfa,
+    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false>, tm_a, tm_b, tm_ao, tm_bo, tm_sfa,
                               tm_sfb, tm_y, a);
   }
   const int sms = device_num_sms();
   const int grid = ntiles < sms ? ntiles : sms;
   const size_t smem = gemm_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (act != nullptr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_dual_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    gemm_dual_kernel<true><<<grid, GEMM_THREADS, smem, stream>>>(tm_a, tm_b, tm_ao, tm_bo, a);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(gemm_dual_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  gemm_dual_kernel<<<grid, GEMM_THREADS, smem, stream>>>(tm_a, tm_b, tm_ao, tm_bo, a);
+  gemm_dual_kernel<false><<<grid, GEMM_THREADS, smem, stream>>>(tm_a, tm_b, tm_ao, tm_bo, a);
   return cudaGetLastError();
 }
 

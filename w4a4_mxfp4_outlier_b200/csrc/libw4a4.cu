@@ -9,3 +9,4 @@
 #include "noalloc.cu"
 #include "checkpoint.cu"
 #include "metrics.cu"
+#include "ffn.cu"

@@ -20,7 +20,8 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
                                                      const int32_t* __restrict__ jmap, int kj,
                                                      int nblk, int d_out, int sfb_rows, int layout,
                                                      uint8_t* __restrict__ wq,
-                                                     uint8_t* __restrict__ sfb) {
+                                                     uint8_t* __restrict__ sfb,
+                                                     const int32_t* __restrict__ rows) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int groups = sfb_rows / 32;
@@ -29,6 +30,7 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
   const int b = warp % nblk;
   const int n = g * 32 + lane;
   const bool row_ok = n < d_out;
+  const int64_t src_row = row_ok ? (rows ? rows[n] : n) : 0;
   float v[32];
   float amax = 0.f;
 #pragma unroll
@@ -37,8 +39,7 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
     float x = 0.f;
     if (row_ok && p < kj) {
       const int j = jmap[p];
-      x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[static_cast<int64_t>(n) * ldw + j]) << 16),
-                    s[j]);
+      x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[src_row * ldw + j]) << 16), s[j]);
     }
     v[i] = x;
     amax = fmaxf(amax, fabsf(x));
@@ -66,7 +67,8 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
 // W_hp[n, i] = bf16_rn(fl32(W[n, O[i]] * s[O[i]])) for i < k, 0 for k <= i < k_pad.
 __global__ void pack_o_kernel(const uint16_t* __restrict__ W, int64_t ldw,
                               const float* __restrict__ s, const int32_t* __restrict__ O, int k,
-                              int k_pad, int d_out, __nv_bfloat16* __restrict__ w_hp) {
+                              int k_pad, int d_out, __nv_bfloat16* __restrict__ w_hp,
+                              const int32_t* __restrict__ rows) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<int64_t>(d_out) * k_pad) return;
   const int n = static_cast<int>(idx / k_pad);
@@ -74,15 +76,15 @@ __global__ void pack_o_kernel(const uint16_t* __restrict__ W, int64_t ldw,
   float x = 0.f;
   if (i < k) {
     const int j = O[i];
-    x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[static_cast<int64_t>(n) * ldw + j]) << 16),
-                  s[j]);
+    const int64_t src_row = rows ? rows[n] : n;
+    x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[src_row * ldw + j]) << 16), s[j]);
   }
   w_hp[idx] = __float2bfloat16_rn(x);
 }
 
 cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,
                         const int32_t* jmap, const Geometry& g, int layout, uint8_t* wq,
-                        uint8_t* sfb, void* w_hp, cudaStream_t stream) {
+                        uint8_t* sfb, void* w_hp, cudaStream_t stream, const int32_t* rows) {
   if (layout == W4A4_SF_32x1_KMAJOR || layout == W4A4_SF_128x1_KMAJOR) {
     // 32x1 / 128x1 stripes: the fold w * s_j, the compaction, the per-row
     // block encoding and the bf16 outlier columns are exactly what the
@@ -94,7 +96,7 @@ cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_
       if (e != cudaSuccess) return e;
     }
     return launch_prep(W, g.d_out, ldw, s, O, jmap, g, wq, sfb, w_hp, stream,
-                       layout == W4A4_SF_128x1_KMAJOR);
+                       layout == W4A4_SF_128x1_KMAJOR, rows);
   }
   if (g.nblk > 0) {
     const int64_t warps = (g.sfb_rows / 32) * g.nblk;
@@ -102,7 +104,7 @@ cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_
     pack_j_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const uint16_t*>(W), ldw, s, jmap, static_cast<int>(g.kj),
         static_cast<int>(g.nblk), static_cast<int>(g.d_out), static_cast<int>(g.sfb_rows), layout,
-        wq, sfb);
+        wq, sfb, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -110,7 +112,7 @@ cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_
     const int64_t total = g.d_out * g.k_pad;
     pack_o_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
         static_cast<const uint16_t*>(W), ldw, s, O, static_cast<int>(g.k), static_cast<int>(g.k_pad),
-        static_cast<int>(g.d_out), static_cast<__nv_bfloat16*>(w_hp));
+        static_cast<int>(g.d_out), static_cast<__nv_bfloat16*>(w_hp), rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -51,7 +51,7 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
                 const float* __restrict__ inv_s, const int32_t* __restrict__ O,
                 const int32_t* __restrict__ jmap, int k, int k_pad, int kj, int nchunks, int nblk,
                 uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa, uint32_t* __restrict__ xo,
-                int stripe4) {
+                int stripe4, const int32_t* __restrict__ rows) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kPrepStages) * kPrepStage);
   uint64_t* empty = full + kPrepStages;
@@ -90,7 +90,10 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
         break;
       if (elect_one()) {
         mbar_arrive_expect_tx(&full[u], bytes);
-        bulk_load(smem + static_cast<size_t>(u) * kPrepStage, src, bytes, &full[u]);
+        // output row r reads input row rows[r] when a row map is given
+        const uint16_t* from =
+            rows ? X + static_cast<int64_t>(rows[blockIdx.x + i * gridDim.x]) * ldx : src;
+        bulk_load(smem + static_cast<size_t>(u) * kPrepStage, from, bytes, &full[u]);
       }
       __syncwarp();
       src += src_step;
@@ -270,7 +273,8 @@ template <int CH>
 static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, int64_t T,
                                   int64_t ldx, const float* inv_s, const int32_t* O,
                                   const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                                  uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4) {
+                                  uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4,
+                                  const int32_t* rows) {
   cudaError_t e = cudaFuncSetAttribute(prep_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kPrepSmem));
   if (e != cudaSuccess) return e;
@@ -278,21 +282,22 @@ static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, in
       static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
       static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
       static_cast<int>(g.kj_pad / 8), static_cast<int>(g.nblk), aq, sfa,
-      static_cast<uint32_t*>(xo), stripe4 ? 1 : 0);
+      static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
                         const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4) {
+                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4,
+                        const int32_t* rows) {
   if (T == 0) return cudaSuccess;
   const PrepPlan p = plan_prep(g);
   const int sms = device_num_sms();
   const int grid = static_cast<int>(T < sms ? T : sms);
   switch (p.ch) {
-    case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
-    case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
-    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4);
+    case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
   }
 }
 

@@ -114,6 +114,45 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ---------------------------------------------------------------------------
+// GELU of the FFN between the two projections, float32, one fixed sequence of
+// IEEE operations (each product, sum and quotient rounded on its own, no
+// contraction into FMA), so that the value -- which decides quantised codes
+// downstream -- is reproducible off the GPU:
+//   gelu(x) = x / (1 + exp(z)),  z = clamp(-2 sqrt(2/pi) (x + 0.044715 x^3), -87, 88)
+// exp(z) by Cody-Waite reduction z = n ln2 + r, n = round-half-even(z log2 e),
+// ln2 = LN2_HI (16 significant bits, so n * LN2_HI is exact) + LN2_LO, then
+// the degree-7 Taylor polynomial of exp(r) (|r| <= 0.35) in Horner form
+// times 2^n built from the exponent bits.  Max error of exp <= 2 ulp; of gelu
+// < 1e-6 absolute against the exact tanh form.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ffn_exp(float z) {
+  constexpr float kLog2e = static_cast<float>(1.4426950408889634);
+  constexpr float kLn2Hi = 0.693145751953125f;
+  constexpr float kLn2Lo = static_cast<float>(1.428606765330187e-06);
+  const float n = rintf(__fmul_rn(z, kLog2e));
+  const float r = __fsub_rn(__fsub_rn(z, __fmul_rn(n, kLn2Hi)), __fmul_rn(n, kLn2Lo));
+  float p = static_cast<float>(1.0 / 5040.0);
+  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 720.0));
+  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 120.0));
+  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 24.0));
+  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 6.0));
+  p = __fadd_rn(__fmul_rn(p, r), 0.5f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  const float scale = __int_as_float((static_cast<int>(n) + 127) << 23);
+  return __fmul_rn(p, scale);
+}
+
+__device__ __forceinline__ float ffn_gelu(float x) {
+  constexpr float kA = static_cast<float>(-2.0 * 0.7978845608028654);
+  constexpr float kB = static_cast<float>(0.044715);
+  const float x3 = __fmul_rn(__fmul_rn(x, x), x);
+  float z = __fmul_rn(kA, __fadd_rn(x, __fmul_rn(kB, x3)));
+  z = fminf(fmaxf(z, -87.0f), 88.0f);
+  return __fdiv_rn(x, __fadd_rn(1.0f, ffn_exp(z)));
+}
+
+// ---------------------------------------------------------------------------
 // TMA and bulk copies (global -> shared, completion counted on an mbarrier)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

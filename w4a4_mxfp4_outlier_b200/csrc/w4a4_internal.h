@@ -49,16 +49,31 @@ cudaError_t launch_finalize(const float* act, const float* wsc, int d_in, double
                             float* s, float* inv_s, float* score, int32_t* O, int32_t* jmap,
                             cudaStream_t stream);
 int finalize_max_d();
+// rows (optional, device int32 [d_out]): packed row n is W row rows[n]
 cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,
                         const int32_t* jmap, const Geometry& g, int layout, uint8_t* wq,
-                        uint8_t* sfb, void* w_hp, cudaStream_t stream);
-// stripe4 = true: one exponent per 4 consecutive blocks (128x1 weight stripes)
+                        uint8_t* sfb, void* w_hp, cudaStream_t stream,
+                        const int32_t* rows = nullptr);
+// stripe4 = true: one exponent per 4 consecutive blocks (128x1 weight stripes);
+// rows (optional, device int32 [T]): output row r reads input row rows[r].
 cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,
                         const int32_t* O, const int32_t* jmap, const Geometry& g, uint8_t* aq,
-                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4 = false);
+                        uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4 = false,
+                        const int32_t* rows = nullptr);
 bool prep_supported(const Geometry& g);
+// Outputs of the fused FFN epilogue: the next layer's activation buffers
+// (Aq, SFA, X_O) and its inv_s in this layer's output-column order.
+struct ActOut {
+  const float* inv_s;
+  uint8_t* aq;
+  uint8_t* sfa;
+  void* xo;
+  int64_t kj, nblk, k_pad;
+};
+// act == nullptr: Y = bf16 product.  Otherwise Y is not written and the
+// product feeds `act` (see GemmArgs in gemm.cu).
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
                         const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
-                        void* Y, int64_t ldy, cudaStream_t stream);
+                        void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act = nullptr);
 
 }  // namespace w4a4

@@ -40,6 +40,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "dual-branch W4A4 GEMM TFLOPS & % of FP4 peak; prep kernel HBM GB/s"
+LAYOUT_NAMES = {0: "32x1", 1: "32x32", 2: "128x1"}
 FP4_NOMINAL_TFLOPS = 9000.0        # B200 dense FP4, datasheet
 FP4_PER_BF16 = 4.0                 # nominal dense FP4 : BF16 ratio (9 / 2.25 PFLOP/s)
 HBM_NOMINAL_GBS = 8000.0
@@ -360,7 +361,7 @@ def run_gpu(args):
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
             "config": {"workload": f"{args.workload}: " + ", ".join(
                 f"{L.name} T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
-                f"{'32x32' if L.layout else '32x1'}" for L in layers),
+                f"{LAYOUT_NAMES[L.layout]}" for L in layers),
                 "tokens_per_gpu": layers[0].T, "parallelism": f"token shards x{world}",
                 "l2": "inputs larger than L2 (no flush)",
                 "step": "calib absmax X,W + finalize + pack + prep + dual GEMM per layer"},
@@ -518,6 +519,131 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_ffn(args):
+    """The FFN pair at T=57600 (Wan2.2 block: 5120 -> 13824, GELU, 13824 -> 5120)
+    with the down layer fed by the up layer's output.  Both layers are
+    calibrated and packed before the timed region; a step is the online
+    forward of one batch: fused (prep, up GEMM whose epilogue writes the down
+    layer's quantised activations, down GEMM) and, timed after it for
+    comparison, unfused (up linear to bf16 Y, GELU, down linear)."""
+    import torch
+
+    import synth
+    import w4a4_mxfp4_outlier_b200 as w4
+    from w4a4_mxfp4_outlier_b200 import ffn
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    active = dist_init("nccl", world, rank)
+    Lu, Ld = synth.FULL_UP.with_(seed=1000 * rank), synth.FULL_DOWN
+    T, d_model, d_ff = Lu.T, Lu.d_in, Lu.d_out
+    X, W_up = synth.gen_layer(Lu, device)
+    W_down = synth.gen_w(Ld.w, Ld.d_out, Ld.d_in, seed=Ld.seed + 1 + 1000 * rank, device=device)
+    f = ffn.calibrate_ffn(X, W_up, W_down, Lu.alpha, Lu.k, Ld.alpha, Ld.k, Lu.layout)
+    act_up, act_down = w4.alloc_act(T, f.up), w4.alloc_act(T, f.down)
+    Y = torch.empty((T, d_model), dtype=torch.bfloat16, device=device)
+    ws_u = torch.empty(w4.workspace_size(T, d_model, d_ff, Lu.k), dtype=torch.uint8, device=device)
+    ws_d = torch.empty(w4.workspace_size(T, d_ff, d_model, Ld.k), dtype=torch.uint8, device=device)
+    Yu = torch.empty((T, d_ff), dtype=torch.bfloat16, device=device)
+    H = torch.empty((T, d_ff), dtype=torch.bfloat16, device=device)
+    Y2 = torch.empty_like(Y)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+
+    def fused(ev=None):
+        if ev: ev[0].record()
+        w4.prep_act(X, f.up, act_up)
+        if ev: ev[1].record()
+        ffn.gemm_dual_act(act_up, T, f, act_down)
+        if ev: ev[2].record()
+        w4.gemm_dual(act_down, T, f.down, Y)
+        if ev: ev[3].record()
+        return 3
+
+    def unfused():
+        w4.linear(X, f.up_plain, ws_u, Yu)
+        ffn.gelu_bf16(Yu, H)
+        w4.linear(H, f.down, ws_d, Y2)
+
+    for _ in range(args.warmup):
+        fused()
+        unfused()
+    st, bits = w4.last_error()
+    if st != w4.OK:
+        raise RuntimeError(f"device error word {bits:#x} during warm-up")
+    if not torch.equal(Y.view(torch.int16), Y2.view(torch.int16)):
+        raise RuntimeError("fused and unfused FFN outputs differ")
+
+    evs = [[mk() for _ in range(4)] for _ in range(args.steps)]
+    t0, t1, u0, u1 = mk(), mk(), mk(), mk()
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    dist_barrier(active, device)
+    clocks.start()
+    time.sleep(0.2)
+    clocks.mark_start()
+    t0.record()
+    launches = 0
+    for k in range(args.steps):
+        launches += fused(evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    clock_info = clocks.stop()
+    u0.record()
+    for _ in range(args.steps):
+        unfused()
+    u1.record()
+    torch.cuda.synchronize()
+    dist_barrier(active, device)
+    step_ms = t0.elapsed_time(t1) / args.steps
+    step_ms_max = dist_max(step_ms, active, device)
+    unfused_ms = u0.elapsed_time(u1) / args.steps
+    flops = 2.0 * (2.0 * T * d_model * d_ff)
+    value = aggregate(flops, world, step_ms_max * 1e-3) / 1e12
+    avg = lambda i, j: sum(e[i].elapsed_time(e[j]) for e in evs) / args.steps
+    prep_ms, up_ms, down_ms = avg(0, 1), avg(1, 2), avg(2, 3)
+    gemm_tflops = flops / ((up_ms + down_ms) * 1e-3) / 1e12
+    peaks, src = measured_peaks()
+    boost = (clock_info.get("sm_mhz") and clock_info.get("sm_max_mhz")
+             and clock_info["sm_mhz"] >= 0.95 * clock_info["sm_max_mhz"])
+    key = "bf16_tflops" if boost else "bf16_tflops_sustained"
+    fp4_peak = peaks[key] * FP4_PER_BF16
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
+            "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
+            "config": {"workload": f"ffn: T={T} {d_model}->{d_ff} k={Lu.k} alpha={Lu.alpha}, GELU, "
+                                   f"{d_ff}->{d_model} k={Ld.k} alpha={Ld.alpha}, "
+                                   f"{LAYOUT_NAMES[Lu.layout]}",
+                       "tokens_per_gpu": T, "parallelism": f"token shards x{world}",
+                       "l2": "inputs larger than L2 (no flush)",
+                       "step": "online FFN forward, fused: prep + up GEMM with GELU/prep epilogue "
+                               "+ down GEMM (packed weights prepared before timing)"},
+            "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+                         "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                         "kernel": "gemm_dual_pair_kernel (up with fused epilogue, down)",
+                         "peak_source": f"{src}: {key} x {FP4_PER_BF16:g}, of measured"},
+            "cpu_baseline": None,
+            "e2e": None,
+            "gpu_launches": launches,
+            "clocks": clock_info,
+            "kernels": {"prep_ms": round(prep_ms, 4), "up_gemm_fused_ms": round(up_ms, 4),
+                        "down_gemm_ms": round(down_ms, 4), "gemm_tflops": round(gemm_tflops, 1),
+                        "unfused_ms_per_step": round(unfused_ms, 4),
+                        "fused_speedup": round(unfused_ms / step_ms, 3),
+                        "outputs_bit_identical": True},
+        }
+        print(json.dumps(out), flush=True)
+    if active:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -525,7 +651,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="full",
                     choices=["full", "full_up", "full_down", "mid_up", "mid_down", "ffn0", "ffn2", "tiny",
-                             "sweep"])
+                             "sweep", "ffn"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -533,6 +659,8 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)      # at least three untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "ffn":
+        run_ffn(args)
     else:
         run_gpu(args)
 

@@ -88,18 +88,41 @@ struct GemmArgs {
   int act_kj, act_nblk, act_k_pad;
 };
 
-// One lane's 32 accumulator columns col0 .. col0+31 of row `row` through the
-// fused FFN epilogue (see GemmArgs).  No warp collectives: callable per lane.
-__device__ __forceinline__ void act_block(const uint32_t (&acc)[32], int row, int col0,
+// Accumulator columns as bf16 pairs: the first step of the fused epilogue
+// (bf16(acc), as the plain epilogue would store it), done right after the
+// tensor-memory load so the pairs take half the registers.
+__device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], uint32_t (&yb)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const __nv_bfloat162 b2 =
+        __floats2bfloat162_rn(__uint_as_float(acc[2 * j]), __uint_as_float(acc[2 * j + 1]));
+    yb[j] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+}
+
+// One lane's 32 columns col0 .. col0+31 of row `row` (as bf16 pairs) through
+// the fused FFN epilogue (see GemmArgs).  No warp collectives: callable per lane.
+__device__ __forceinline__ void act_block(const uint32_t (&yb)[16], int row, int col0,
                                           const GemmArgs& a) {
   if (row >= a.T) return;
   float v[32];
+  const bool full = col0 + 32 <= a.d_out;   // d_out % 16 == 0: a chunk is all in or
+#pragma unroll                               // straddles at 16
+  for (int q = 0; q < 8; ++q) {
+    float4 is = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (full || col0 + 4 * q < a.d_out) is = *reinterpret_cast<const float4*>(a.act_inv_s + col0 + 4 * q);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int col = col0 + i;
-    const float y = __bfloat162float(__float2bfloat16_rn(__uint_as_float(acc[i])));
-    const float x = __bfloat162float(__float2bfloat16_rn(ffn_gelu(y)));
-    v[i] = col < a.d_out ? __fmul_rn(x, a.act_inv_s[col]) : 0.0f;
+    for (int h = 0; h < 2; ++h) {
+      const int i = 4 * q + 2 * h;
+      const float2 y = make_float2(__uint_as_float(yb[i >> 1] << 16),
+                                   __uint_as_float(yb[i >> 1] & 0xFFFF0000u));
+      const float2 g = ffn_gelu_x2(y);
+      const float2 x = make_float2(__bfloat162float(__float2bfloat16_rn(g.x)),
+                                   __bfloat162float(__float2bfloat16_rn(g.y)));
+      const float2 w = __fmul2_rn(x, h ? make_float2(is.z, is.w) : make_float2(is.x, is.y));
+      v[i] = col0 + i < a.d_out ? w.x : 0.0f;
+      v[i + 1] = col0 + i + 1 < a.d_out ? w.y : 0.0f;
+    }
   }
   // outlier columns of the next layer (and its zero padding up to k_pad)
   if (col0 + 32 > a.act_kj && col0 < a.act_kj + a.act_k_pad) {
@@ -328,6 +351,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
       tmem_ld_wait();
+      uint32_t yb[4][16];
+      if constexpr (kAct) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) pack_bf16_pairs(r[c], yb[c]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);
@@ -335,7 +363,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int row = tm * BM + 32 * sp + lane;
       if constexpr (kAct) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(r[c], row, tn * BN + 128 * half + 32 * c, args);
+        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * BN + 128 * half + 32 * c, args);
       } else if (row < args.T) {
         __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
 #pragma unroll
@@ -636,6 +664,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
       tmem_ld_wait();
+      uint32_t yb[4][16];
+      if constexpr (kAct) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) pack_bf16_pairs(r[c], yb[c]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
@@ -643,7 +676,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (kAct) {
         const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(r[c], row, tn * 256 + 128 * half + 32 * c, args);
+        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, args);
         continue;
       }
       // Y through a per-warp staging block, 16 rows x 32 columns at a time:

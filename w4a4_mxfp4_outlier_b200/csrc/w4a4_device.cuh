@@ -152,6 +152,39 @@ __device__ __forceinline__ float ffn_gelu(float x) {
   return __fdiv_rn(x, __fadd_rn(1.0f, ffn_exp(z)));
 }
 
+// The same two functions on a pair of values with the packed float32x2
+// operations (each lane of a packed op rounds exactly as the scalar op does,
+// so results are identical to ffn_exp / ffn_gelu element by element).
+__device__ __forceinline__ float2 ffn_exp_x2(float2 z) {
+  constexpr float kLog2e = static_cast<float>(1.4426950408889634);
+  constexpr float kLn2Hi = 0.693145751953125f;
+  constexpr float kLn2Lo = static_cast<float>(1.428606765330187e-06);
+  const float2 t = __fmul2_rn(z, make_float2(kLog2e, kLog2e));
+  const float2 n = make_float2(rintf(t.x), rintf(t.y));
+  const float2 r = __fadd2_rn(__fadd2_rn(z, __fmul2_rn(n, make_float2(-kLn2Hi, -kLn2Hi))),
+                              __fmul2_rn(n, make_float2(-kLn2Lo, -kLn2Lo)));
+  float2 p = make_float2(static_cast<float>(1.0 / 5040.0), static_cast<float>(1.0 / 5040.0));
+  const float c[7] = {static_cast<float>(1.0 / 720.0), static_cast<float>(1.0 / 120.0),
+                      static_cast<float>(1.0 / 24.0),  static_cast<float>(1.0 / 6.0),
+                      0.5f, 1.0f, 1.0f};
+#pragma unroll
+  for (int i = 0; i < 7; ++i) p = __fadd2_rn(__fmul2_rn(p, r), make_float2(c[i], c[i]));
+  const float2 scale = make_float2(__int_as_float((static_cast<int>(n.x) + 127) << 23),
+                                   __int_as_float((static_cast<int>(n.y) + 127) << 23));
+  return __fmul2_rn(p, scale);
+}
+
+__device__ __forceinline__ float2 ffn_gelu_x2(float2 x) {
+  constexpr float kA = static_cast<float>(-2.0 * 0.7978845608028654);
+  constexpr float kB = static_cast<float>(0.044715);
+  const float2 x3 = __fmul2_rn(__fmul2_rn(x, x), x);
+  float2 z = __fmul2_rn(make_float2(kA, kA), __fadd2_rn(x, __fmul2_rn(make_float2(kB, kB), x3)));
+  z.x = fminf(fmaxf(z.x, -87.0f), 88.0f);
+  z.y = fminf(fmaxf(z.y, -87.0f), 88.0f);
+  const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), ffn_exp_x2(z));
+  return make_float2(__fdiv_rn(x.x, d.x), __fdiv_rn(x.y, d.y));
+}
+
 // ---------------------------------------------------------------------------
 // TMA and bulk copies (global -> shared, completion counted on an mbarrier)
 // ---------------------------------------------------------------------------

@@ -186,9 +186,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "392bb6a4ca7679722ed6fb15ce83149887ed331b22eea44e0fe922733e2b5345",
+    "sha256": "6aa35026cdb7bf54ff41c662e438cd1c225aaabc42485e0d472f50a59bf3554f",
     "workload": "full",
-    "bytes_per_launch": (728140288 + 1555996928 + 1510572032 + 571407872) / 2,
+    "bytes_per_launch": (750766336 + 1558680832 + 1657089536 + 572224256) / 2,
 }
 
 

@@ -89,53 +89,95 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 # The review quantises both FFN projections of the Wan2.2 DiT (ffn.0 and
 # ffn.2, §3.1/§3.5); between them the FFN applies GELU (tanh form), which the
 # pages do not write out.  The fused up->down step feeds the down projection
-# with X_down = bf16_rn(gelu(bf16 Y_up)).  Because the GELU value decides
-# quantised codes, the oracle takes that decision in the kernel's precision,
-# float32, with one fixed sequence of IEEE operations (every product, sum and
-# quotient separately rounded, no fused multiply-add):
+# with X_down = bf16_rn(gelu(y)) for the bf16 value y = bf16(Y_up): the bf16
+# number nearest the exact value
 #
-#   gelu(x) = x / (1 + exp(z)),  z = clamp(-2 * 0.7978845608 * (x + 0.044715 x^3), -87, 88)
+#   gelu(y) = 0.5 y (1 + tanh(u)) = y / (1 + exp(-2u)),  u = sqrt(2/pi) (y + 0.044715 y^3),
 #
-# (0.5 x (1 + tanh(u)) = x / (1 + exp(-2u))), with exp by Cody-Waite range
-# reduction z = n ln2 + r (n = round-half-even(z log2 e), ln2 split into a
-# high part exact in 16 bits and a low part) and the degree-7 Taylor
-# polynomial of exp(r) on |r| <= 0.35 in Horner form, times 2^n.
+# ties to even.  That is a function of the 16-bit input with a plain
+# definition, so it does not depend on how a kernel evaluates it.  The oracle
+# evaluates the second form in float64 (no cancellation for negative y) and
+# rounds that once to bf16.  Where the float64 value lies so close to a bf16
+# rounding boundary that its own error could decide the rounding (it happens
+# for the smallest inputs: gelu(y) = y/2 + O(y^2) with y/2 a bf16 midpoint),
+# it recomputes the value with 100 significant digits and decides by exact
+# comparison with the boundary (the usual correct-rounding strategy).
 
-_F = np.float32
-_LOG2E = _F(1.4426950408889634)
-_LN2_HI = _F(0.693145751953125)          # 0x3F317200: 16 significant bits, n * LN2_HI exact
-_LN2_LO = _F(1.428606765330187e-06)      # ln 2 - LN2_HI
-_EXP_C = [_F(1.0 / 5040), _F(1.0 / 720), _F(1.0 / 120), _F(1.0 / 24), _F(1.0 / 6), _F(0.5),
-          _F(1.0), _F(1.0)]               # Horner order, highest degree first
-_GELU_A = _F(-2.0 * 0.7978845608028654)  # -2 sqrt(2 / pi)
-_GELU_B = _F(0.044715)
+_SQRT_2_OVER_PI = np.sqrt(2.0 / np.pi)
 
 
-def exp_f32(z: np.ndarray) -> np.ndarray:
-    """exp of float32 z in [-87, 88] by the steps above (float32 arithmetic)."""
-    z = np.asarray(z, dtype=np.float32)
-    n = np.rint(z * _LOG2E).astype(np.float32)                   # ties to even
-    r = (z - n * _LN2_HI) - n * _LN2_LO
-    p = np.full_like(r, _EXP_C[0])
-    for c in _EXP_C[1:]:
-        p = p * r + c
-    scale = ((n.astype(np.int32) + 127).astype(np.uint32) << 23).view(np.float32)
-    return (p * scale).astype(np.float32)
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float64 -> bfloat16 bit patterns, round to nearest, ties to even, in one
+    step (no intermediate float32 rounding).  bf16 keeps 8 significant bits
+    down to 2^-126 and a fixed quantum of 2^-133 below (subnormals)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        _, e = np.frexp(a)                                 # a = m 2^e, m in [0.5, 1)
+        E = np.maximum(e.astype(np.int64) - 1, -126)       # binade exponent, floored at the subnormals
+        q = np.ldexp(1.0, (E - 7).astype(np.int32))        # quantum of that binade
+        n = np.rint(a / q)                                 # exact scaling; rint ties to even
+        v = n * q
+        v = np.where(v > 3.3895313892515355e38, np.inf, v)   # beyond the largest bf16: inf
+        v = np.where(np.isfinite(a), v, a)
+        v = np.where(a == 0.0, 0.0, v)
+    r = np.copysign(v, x).astype(np.float32)               # exact: v is a bf16 value
+    bits = (r.view(np.uint32) >> 16).astype(np.uint16)
+    return np.where(np.isnan(x), np.uint16(0x7FC0), bits)
 
 
-def gelu_f32(x: np.ndarray) -> np.ndarray:
-    """GELU (tanh form) of float32 x, as defined above."""
-    x = np.asarray(x, dtype=np.float32)
-    with np.errstate(over="ignore", invalid="ignore"):      # |x|^3 may overflow to inf
-        x3 = (x * x) * x
-        z = _GELU_A * (x + _GELU_B * x3)
-        z = np.minimum(np.maximum(z, _F(-87.0)), _F(88.0))
-        return (x / (_F(1.0) + exp_f32(z))).astype(np.float32)
+def _bf16_quantum(a: np.ndarray) -> np.ndarray:
+    """Spacing of the bf16 values around |a| > 0 (2^-133 below 2^-126)."""
+    _, e = np.frexp(a)
+    return np.ldexp(1.0, (np.maximum(e.astype(np.int64) - 1, -126) - 7).astype(np.int32))
+
+
+def _gelu_bf16_exact(yv: float) -> int:
+    """bf16 bits of gelu(yv), decided with 100-digit arithmetic."""
+    import mpmath
+    with mpmath.workdps(100):
+        y = mpmath.mpf(yv)
+        u = mpmath.sqrt(2 / mpmath.pi) * (y + mpmath.mpf("0.044715") * y ** 3)
+        g = y / (1 + mpmath.exp(-2 * u))
+        a = abs(g)
+        q = mpmath.mpf(float(_bf16_quantum(np.array([float(a)]))[0]))
+        n = int(mpmath.floor(a / q))
+        mid = (n + mpmath.mpf(0.5)) * q
+        if a > mid or (a == mid and n % 2 == 1):
+            n += 1
+        v = float(n * q)                         # exact: a bf16 value
+    return int(f64_to_bf16_bits(np.array([-v if g < 0 or (g == 0 and yv < 0) else v]))[0])
+
+
+def gelu_bf16(y: np.ndarray) -> np.ndarray:
+    """bf16_rn(gelu(y)) for bf16-exact float32 y, as float32 (see above).
+    Non-finite inputs follow the float64 formula: +inf -> +inf, -inf and NaN
+    -> NaN."""
+    yf = np.asarray(y, dtype=np.float32)
+    yd = yf.astype(np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        u = _SQRT_2_OVER_PI * (yd + 0.044715 * (yd * yd * yd))
+        g = yd / (1.0 + np.exp(-2.0 * u))
+    bits = f64_to_bf16_bits(g)
+    # float64 carries ~2^-45 of a bf16 quantum of error here; look again at
+    # every value within 2^-20 quanta of a rounding boundary
+    a = np.abs(g)
+    check = np.isfinite(a) & (a > 0) & (a < 3.3e38)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        frac = np.where(check, a / np.where(check, _bf16_quantum(np.where(check, a, 1.0)), 1.0), 0.0)
+    near = check & (np.abs(frac - np.floor(frac) - 0.5) < 2.0 ** -20)
+    if near.any():
+        flat_bits = bits.reshape(-1)
+        flat_y = yd.reshape(-1)
+        for i in np.flatnonzero(near.reshape(-1)):
+            flat_bits[i] = _gelu_bf16_exact(float(flat_y[i]))
+        bits = flat_bits.reshape(bits.shape)
+    return bf16_bits_to_f32(bits)
 
 
 def ffn_hidden(Y_up: np.ndarray) -> np.ndarray:
     """X_down = bf16_rn(gelu(Y_up)) for bf16-exact float32 Y_up."""
-    return bf16_bits_to_f32(f32_to_bf16_bits(gelu_f32(Y_up)))
+    return gelu_bf16(Y_up)
 
 
 # ----------------------------------------------------------------------------

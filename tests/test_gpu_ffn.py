@@ -4,9 +4,9 @@ up-projection epilogue against the oracle; fused and unfused FFN outputs.
 The fused epilogue is checked bit for bit against the oracle applied to the
 GPU's own (unfused) up-layer output: bf16(acc) is the same value in both
 GPU paths (one kernel main loop, the epilogue differs), so from there every
-step -- GELU in float32, bf16 rounding, the multiply by inv_s, the MXFP4
-encoding -- is a deterministic float32 or integer decision both sides take
-alike."""
+step -- the correctly rounded bf16 GELU, the multiply by inv_s, the MXFP4
+encoding -- is a function of that value (a rounding, a float32 product, an
+integer decision) that both sides compute alike."""
 import numpy as np
 import pytest
 import torch
@@ -31,7 +31,7 @@ def test_gelu_every_bf16():
     Y = torch.from_numpy(x[:n].reshape(-1, 64)).to(torch.bfloat16).cuda()
     H = ffn.gelu_bf16(Y)
     torch.cuda.synchronize()
-    ref = orc.f32_to_bf16_bits(orc.gelu_f32(x[:n])).reshape(-1, 64)
+    ref = orc.f32_to_bf16_bits(orc.gelu_bf16(x[:n])).reshape(-1, 64)
     np.testing.assert_array_equal(gu.bf16_bits(H), ref)
 
 

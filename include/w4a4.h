@@ -236,12 +236,11 @@ w4a4_status w4a4_packed_load(const void* host, size_t bytes, const w4a4_packed_w
 /* ------------------------------------------------------------------------
  * The FFN pair (review sec. 3.1, 3.5: both FFN projections, ffn.0 up and
  * ffn.2 down, take the same W4A4 recipe).  Between them the Wan2.2 FFN
- * applies GELU, which the pages do not write out; here X_down =
- * bf16_rn(gelu(bf16 Y_up)) with GELU in tanh form evaluated in float32 by a
- * fixed sequence of IEEE operations: gelu(x) = x / (1 + exp(z)), z =
- * clamp(-2 sqrt(2/pi) (x + 0.044715 x^3), -87, 88), exp by Cody-Waite
- * reduction and a degree-7 Taylor polynomial (|error| < 1e-6 against the
- * exact tanh form).
+ * applies GELU, which the pages do not write out; here X_down[t, c] is the
+ * bf16 value nearest (ties to even) the exact GELU in tanh form,
+ * gelu(y) = 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))), of the bf16
+ * value y = bf16_rn(Y_up[t, c]): a function of the 16-bit input, the same
+ * whether fused or not.  +inf maps to +inf, -inf and NaN to NaN.
  *
  * Fused use: calibrate and pack the down layer, w4a4_ffn_link it, pack the up
  * weight with w4a4_pack_weight_rows(rows = perm), then per batch
@@ -250,8 +249,9 @@ w4a4_status w4a4_packed_load(const void* host, size_t bytes, const w4a4_packed_w
  * ------------------------------------------------------------------------ */
 
 /* X[t, j] = bf16_rn(gelu(Y[t, j])) for a bf16 [T, d] matrix (row strides
- * ldy, ldx elements); the unfused activation, e.g. to calibrate the down
- * layer. */
+ * ldy, ldx elements; X may be Y); the unfused activation, e.g. to calibrate
+ * the down layer.  Errors: INVALID_ARG for negative sizes, ld < d or a null
+ * pointer with T, d > 0. */
 w4a4_status w4a4_gelu_bf16(const void* Y, int64_t T, int64_t d, int64_t ldy, void* X, int64_t ldx,
                            void* stream);
 

@@ -154,8 +154,8 @@ def gelu_bf16(y: np.ndarray) -> np.ndarray:
     Non-finite inputs follow the float64 formula: +inf -> +inf, -inf and NaN
     -> NaN."""
     yf = np.asarray(y, dtype=np.float32)
-    yd = yf.astype(np.float64)
-    with np.errstate(over="ignore", invalid="ignore"):
+    with np.errstate(over="ignore", invalid="ignore"):         # signalling NaNs warn on widening
+        yd = yf.astype(np.float64)
         u = _SQRT_2_OVER_PI * (yd + 0.044715 * (yd * yd * yd))
         g = yd / (1.0 + np.exp(-2.0 * u))
     bits = f64_to_bf16_bits(g)

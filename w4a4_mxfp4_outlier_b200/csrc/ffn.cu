@@ -17,14 +17,46 @@
 
 namespace w4a4 {
 
-// X = bf16(gelu(Y)) elementwise (the unfused form of the FFN activation).
-__global__ void gelu_bf16_kernel(const __nv_bfloat16* __restrict__ Y, int64_t ldy,
-                                 __nv_bfloat16* __restrict__ X, int64_t ldx, int64_t T, int64_t d) {
+// X = bf16(gelu(Y)) elementwise (the unfused form of the FFN activation),
+// with the same table and closed forms the fused GEMM epilogue uses.  Rows of
+// 8-element multiples at 16-byte alignment (`vec`) move as 16-byte vectors,
+// two per thread in flight; anything else goes element by element.
+__device__ __forceinline__ uint32_t gelu_pair(uint32_t tab, uint32_t p) {
+  return gelu_bf16(tab, p & 0xFFFFu) | (gelu_bf16(tab, p >> 16) << 16);
+}
+
+__device__ __forceinline__ uint4 gelu_vec8(uint32_t tab, uint4 v) {
+  return make_uint4(gelu_pair(tab, v.x), gelu_pair(tab, v.y), gelu_pair(tab, v.z), gelu_pair(tab, v.w));
+}
+
+__global__ void __launch_bounds__(512) gelu_bf16_kernel(const uint16_t* __restrict__ Y, int64_t ldy,
+                                                        uint16_t* __restrict__ X, int64_t ldx,
+                                                        int64_t T, int64_t d, int vec) {
+  __shared__ __align__(16) uint16_t tab[kGeluTabEntries];
+  gelu_table_fill(tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const uint32_t tab_s = smem_u32(tab);
+  if (vec) {
+    const int64_t nv = d >> 3;
+    const int64_t bd = blockDim.x;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+      const uint4* y = reinterpret_cast<const uint4*>(Y + t * ldy);
+      uint4* x = reinterpret_cast<uint4*>(X + t * ldx);
+      for (int64_t j = threadIdx.x; j < nv; j += 2 * bd) {
+        const bool two = j + bd < nv;
+        const uint4 a = y[j];
+        const uint4 b = two ? y[j + bd] : make_uint4(0u, 0u, 0u, 0u);
+        x[j] = gelu_vec8(tab_s, a);
+        if (two) x[j + bd] = gelu_vec8(tab_s, b);
+      }
+    }
+    return;
+  }
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    const __nv_bfloat16* y = Y + t * ldy;
-    __nv_bfloat16* x = X + t * ldx;
+    const uint16_t* y = Y + t * ldy;
+    uint16_t* x = X + t * ldx;
     for (int64_t j = threadIdx.x; j < d; j += blockDim.x)
-      x[j] = __float2bfloat16_rn(ffn_gelu(__bfloat162float(y[j])));
+      x[j] = static_cast<uint16_t>(gelu_bf16(tab_s, y[j]));
   }
 }
 
@@ -49,9 +81,11 @@ extern "C" w4a4_status w4a4_gelu_bf16(const void* Y, int64_t T, int64_t d, int64
   if (T == 0 || d == 0) return W4A4_OK;
   if (Y == nullptr || X == nullptr) return W4A4_ERR_INVALID_ARG;
   const int64_t sms = device_num_sms() > 0 ? device_num_sms() : 148;
-  const int64_t grid = T < 8 * sms ? T : 8 * sms;
-  gelu_bf16_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(Y), ldy, static_cast<__nv_bfloat16*>(X), ldx, T, d);
+  // every CTA first fills its own table, so keep the grid to about two per SM
+  const int64_t grid = T < 2 * sms ? T : 2 * sms;
+  const int vec = ((d | ldy | ldx) & 7) == 0 && aligned16(Y) && aligned16(X);
+  gelu_bf16_kernel<<<static_cast<unsigned>(grid), 512, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(Y), ldy, static_cast<uint16_t*>(X), ldx, T, d, vec);
   return cudaGetLastError() == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 

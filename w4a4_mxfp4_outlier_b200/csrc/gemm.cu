@@ -55,6 +55,7 @@ constexpr int GROUP_M = 16;                   // tile raster: 16 M tiles per swe
 
 struct GemmSmem {
   uint8_t stage[STAGES][STAGE_BYTES];         // 1024-aligned (each part 1024-aligned)
+  alignas(16) uint16_t gelu_tab[kGeluTabEntries];   // fused FFN epilogue only
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full;
@@ -91,7 +92,12 @@ struct GemmArgs {
 // Accumulator columns as bf16 pairs: the first step of the fused epilogue
 // (bf16(acc), as the plain epilogue would store it), done right after the
 // tensor-memory load so the pairs take half the registers.
-__device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], uint32_t (&yb)[16]) {
+struct BfPairs16 {
+  uint32_t w[16];    // 32 consecutive columns of one row as bf16 pairs (low half: even column)
+};
+
+__device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], BfPairs16& out) {
+  uint32_t (&yb)[16] = out.w;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const __nv_bfloat162 b2 =
@@ -102,27 +108,51 @@ __device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], uint3
 
 // One lane's 32 columns col0 .. col0+31 of row `row` (as bf16 pairs) through
 // the fused FFN epilogue (see GemmArgs).  No warp collectives: callable per lane.
-__device__ __forceinline__ void act_block(const uint32_t (&yb)[16], int row, int col0,
-                                          const GemmArgs& a) {
+// Not inlined: the epilogue calls it for 4 column chunks per tile, and with
+// four inlined copies the epilogue warps' code was large enough to push the
+// producer and MMA warps' instructions out of the instruction cache -- the
+// fused up-projection GEMM then ran at 0.49x the speed of this form
+// (T = 57600, 5120 -> 13824: 3.13 ms inlined, 1.87 ms called).
+__device__ __noinline__ void act_block(const BfPairs16 y, int row, int col0, const GemmArgs* ap,
+                                       uint32_t gelu_tab) {
+  const uint32_t (&yb)[16] = y.w;
+  const GemmArgs& a = *ap;
   if (row >= a.T) return;
-  float v[32];
-  const bool full = col0 + 32 <= a.d_out;   // d_out % 16 == 0: a chunk is all in or
-#pragma unroll                               // straddles at 16
+  // bf16(gelu(y)) of the 32 columns as bf16 pairs: table lookups, with the
+  // inputs outside the table's range (rare) redone afterwards
+  uint32_t hp[16];
+  uint32_t bad = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t lo = yb[j] & 0xFFFFu, hi = yb[j] >> 16;
+    const uint32_t rl = (lo & 0x7FFFu) - kGeluTabBase, rh = (hi & 0x7FFFu) - kGeluTabBase;
+    bad |= rl | rh;
+    hp[j] = gelu_bf16_table(gelu_tab, lo, rl) | (gelu_bf16_table(gelu_tab, hi, rh) << 16);
+  }
+  if (bad >= 2048u) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t lo = yb[j] & 0xFFFFu, hi = yb[j] >> 16;
+      if ((lo & 0x7FFFu) - kGeluTabBase >= 2048u) hp[j] = (hp[j] & 0xFFFF0000u) | gelu_bf16_outside(lo);
+      if ((hi & 0x7FFFu) - kGeluTabBase >= 2048u) hp[j] = (hp[j] & 0xFFFFu) | (gelu_bf16_outside(hi) << 16);
+    }
+  }
+  // v = fl32(x * inv_s) column by column; columns past d_out are +0
+  float2 v[16];
+#pragma unroll
   for (int q = 0; q < 8; ++q) {
     float4 is = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (full || col0 + 4 * q < a.d_out) is = *reinterpret_cast<const float4*>(a.act_inv_s + col0 + 4 * q);
+    if (col0 + 4 * q < a.d_out) is = *reinterpret_cast<const float4*>(a.act_inv_s + col0 + 4 * q);
+    const uint32_t p0 = hp[2 * q], p1 = hp[2 * q + 1];
+    v[2 * q] = __fmul2_rn(make_float2(__uint_as_float(p0 << 16), __uint_as_float(p0 & 0xFFFF0000u)),
+                          make_float2(is.x, is.y));
+    v[2 * q + 1] = __fmul2_rn(make_float2(__uint_as_float(p1 << 16), __uint_as_float(p1 & 0xFFFF0000u)),
+                              make_float2(is.z, is.w));
+  }
+  if (col0 + 32 > a.d_out) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 4 * q + 2 * h;
-      const float2 y = make_float2(__uint_as_float(yb[i >> 1] << 16),
-                                   __uint_as_float(yb[i >> 1] & 0xFFFF0000u));
-      const float2 g = ffn_gelu_x2(y);
-      const float2 x = make_float2(__bfloat162float(__float2bfloat16_rn(g.x)),
-                                   __bfloat162float(__float2bfloat16_rn(g.y)));
-      const float2 w = __fmul2_rn(x, h ? make_float2(is.z, is.w) : make_float2(is.x, is.y));
-      v[i] = col0 + i < a.d_out ? w.x : 0.0f;
-      v[i + 1] = col0 + i + 1 < a.d_out ? w.y : 0.0f;
-    }
+    for (int j = 0; j < 16; ++j)
+      if (col0 + 2 * j >= a.d_out) v[j] = make_float2(0.f, 0.f);   // d_out is even
   }
   // outlier columns of the next layer (and its zero padding up to k_pad)
   if (col0 + 32 > a.act_kj && col0 < a.act_kj + a.act_k_pad) {
@@ -130,27 +160,35 @@ __device__ __forceinline__ void act_block(const uint32_t (&yb)[16], int row, int
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int o = col0 + i - a.act_kj;
-      if (o >= 0 && o < a.act_k_pad) xr[o] = __float2bfloat16_rn(v[i]);
+      const float vi = (i & 1) ? v[i >> 1].y : v[i >> 1].x;
+      if (o >= 0 && o < a.act_k_pad) xr[o] = __float2bfloat16_rn(vi);
     }
   }
   // the MX block of compacted positions col0 .. col0+31 (zeros past act_kj)
   const int b = col0 >> 5;
   if (b < a.act_nblk) {
+    if (col0 + 32 > a.act_kj) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (col0 + i >= a.act_kj) {
+          if (i & 1) v[i >> 1].y = 0.0f;
+          else v[i >> 1].x = 0.0f;
+        }
+      }
+    }
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (col0 + i >= a.act_kj) v[i] = 0.0f;
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
     const uint32_t code = mx_scale_code(amax);
     const float inv = mx_inv_scale(code);
+    const float2 inv2 = make_float2(inv, inv);
     uint32_t w[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q], inv), __fmul_rn(v[8 * q + 1], inv),
-                        __fmul_rn(v[8 * q + 2], inv), __fmul_rn(v[8 * q + 3], inv),
-                        __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
-                        __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
+    for (int q = 0; q < 4; ++q) {
+      const float2 a0 = __fmul2_rn(v[4 * q], inv2), a1 = __fmul2_rn(v[4 * q + 1], inv2);
+      const float2 a2 = __fmul2_rn(v[4 * q + 2], inv2), a3 = __fmul2_rn(v[4 * q + 3], inv2);
+      w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y);
+    }
     *reinterpret_cast<uint4*>(a.act_aq + static_cast<int64_t>(row) * a.act_nblk * 16 + b * 16) =
         make_uint4(w[0], w[1], w[2], w[3]);
     a.act_sfa[sf_offset(row, b, a.act_nblk)] = static_cast<uint8_t>(code);
@@ -171,7 +209,7 @@ template <bool kAct>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
-                     const GemmArgs args) {
+                     const __grid_constant__ GemmArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -334,6 +372,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int ew = warp - 2;                 // 0..7
     const int sp = warp & 3;                 // tensor-memory lane quarter this warp may read
     const int half = ew >> 2;                // column half: 0 -> 0..127, 1 -> 128..255
+    uint32_t gelu_tab = 0;
+    if constexpr (kAct) {
+      gelu_table_fill(sm.gelu_tab, ew * 32 + lane, NUM_EPI_WARPS * 32);
+      named_bar_sync(1, NUM_EPI_WARPS * 32);
+      gelu_tab = smem_u32(sm.gelu_tab);
+    }
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       int tm, tn;
@@ -351,7 +395,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
       tmem_ld_wait();
-      uint32_t yb[4][16];
+      BfPairs16 yb[4];
       if constexpr (kAct) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) pack_bf16_pairs(r[c], yb[c]);
@@ -363,7 +407,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int row = tm * BM + 32 * sp + lane;
       if constexpr (kAct) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * BN + 128 * half + 32 * c, args);
+        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * BN + 128 * half + 32 * c, &args, gelu_tab);
       } else if (row < args.T) {
         __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
 #pragma unroll
@@ -424,7 +468,9 @@ constexpr int P_EPI_BYTES = 16 * 64;          // staging block: 16 rows x 32 bf1
 
 struct PairSmem {
   uint8_t stage[P_STAGES][P_STAGE_BYTES];
-  alignas(1024) uint8_t epi[NUM_EPI_WARPS][P_EPI_BYTES];   // per epilogue warp: Y staging
+  // per epilogue warp: Y staging; the fused FFN epilogue (no Y) keeps its
+  // GELU table here instead
+  alignas(1024) uint8_t epi[NUM_EPI_WARPS][P_EPI_BYTES];
   uint64_t full[P_STAGES];     // leader's counts the bytes of both CTAs
   uint64_t empty[P_STAGES];    // both CTAs: MMA commit, multicast
   uint64_t acc_full;           // both CTAs: MMA commit, multicast
@@ -439,7 +485,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
-                          const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
+                          const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ GemmArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   PairSmem& sm = *reinterpret_cast<PairSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -649,6 +695,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int sp = warp & 3;
     const int half = ew >> 2;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&sm.acc_empty), 0);
+    uint32_t gelu_tab = 0;
+    if constexpr (kAct) {
+      static_assert(sizeof(sm.epi) >= kGeluTabEntries * sizeof(uint16_t), "GELU table space");
+      uint16_t* tab = reinterpret_cast<uint16_t*>(&sm.epi[0][0]);
+      gelu_table_fill(tab, ew * 32 + lane, NUM_EPI_WARPS * 32);
+      named_bar_sync(1, NUM_EPI_WARPS * 32);
+      gelu_tab = smem_u32(tab);
+    }
     uint32_t tcount = 0;
     for (int t = pair; t < ntiles; t += npairs, ++tcount) {
       int tm, tn;
@@ -664,7 +718,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
       tmem_ld_wait();
-      uint32_t yb[4][16];
+      BfPairs16 yb[4];
       if constexpr (kAct) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) pack_bf16_pairs(r[c], yb[c]);
@@ -676,7 +730,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (kAct) {
         const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, args);
+        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, &args, gelu_tab);
         continue;
       }
       // Y through a per-warp staging block, 16 rows x 32 columns at a time:

@@ -114,75 +114,86 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ---------------------------------------------------------------------------
-// GELU of the FFN between the two projections, float32, one fixed sequence of
-// IEEE operations (each product, sum and quotient rounded on its own, no
-// contraction into FMA), so that the value -- which decides quantised codes
-// downstream -- is reproducible off the GPU:
-//   gelu(x) = x / (1 + exp(z)),  z = clamp(-2 sqrt(2/pi) (x + 0.044715 x^3), -87, 88)
-// exp(z) by Cody-Waite reduction z = n ln2 + r, n = round-half-even(z log2 e),
-// ln2 = LN2_HI (16 significant bits, so n * LN2_HI is exact) + LN2_LO, then
-// the degree-7 Taylor polynomial of exp(r) (|r| <= 0.35) in Horner form
-// times 2^n built from the exponent bits.  Max error of exp <= 2 ulp; of gelu
-// < 1e-6 absolute against the exact tanh form.
+// GELU of the FFN between the two projections, for a bf16 input y, as the
+// bf16 value nearest the exact
+//   gelu(y) = 0.5 y (1 + tanh(u)) = y / (1 + exp(-2u)),  u = sqrt(2/pi) (y + 0.044715 y^3)
+// (tanh form), ties to even.  It is a function of 16 bits, so kernels may
+// evaluate it any way that returns that value:
+//  * 2^-12 <= |y| < 16: a 4096-entry table (sign, 16 binades, 128
+//    mantissas) in shared memory, filled per CTA with gelu_bf16_exact;
+//  * |y| < 2^-12: gelu(y) = y/2 + d with 0 < d <= 0.4 y^2, far below half a
+//    bf16 spacing of y/2, so the result is y/2, except that when y/2 falls
+//    exactly between two bf16 values (only below 2^-125) d breaks the tie
+//    toward +inf;
+//  * |y| >= 16: gelu(y) = y (1 - e), e < 1e-137, rounds to y; for y <= -16
+//    |gelu(y)| < 1e-136 rounds to -0.  +inf -> +inf, -inf and NaN -> NaN
+//    (the value of the second form).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float ffn_exp(float z) {
-  constexpr float kLog2e = static_cast<float>(1.4426950408889634);
-  constexpr float kLn2Hi = 0.693145751953125f;
-  constexpr float kLn2Lo = static_cast<float>(1.428606765330187e-06);
-  const float n = rintf(__fmul_rn(z, kLog2e));
-  const float r = __fsub_rn(__fsub_rn(z, __fmul_rn(n, kLn2Hi)), __fmul_rn(n, kLn2Lo));
-  float p = static_cast<float>(1.0 / 5040.0);
-  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 720.0));
-  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 120.0));
-  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 24.0));
-  p = __fadd_rn(__fmul_rn(p, r), static_cast<float>(1.0 / 6.0));
-  p = __fadd_rn(__fmul_rn(p, r), 0.5f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  const float scale = __int_as_float((static_cast<int>(n) + 127) << 23);
-  return __fmul_rn(p, scale);
+constexpr uint32_t kGeluTabExp0 = 115;      // biased exponent of 2^-12
+constexpr int kGeluTabEntries = 4096;       // 2 signs x 16 binades x 128 mantissas
+constexpr uint32_t kGeluTabBase = kGeluTabExp0 << 7;
+
+// float64 -> bf16 bits, round to nearest even, in one rounding: truncate to
+// float32 and set its last bit if anything was cut off (round to odd keeps
+// the information a second rounding to 8 bits needs), then round to bf16
+__device__ __forceinline__ uint32_t f64_to_bf16_rn(double g) {
+  float f = __double2float_rz(g);
+  if (static_cast<double>(f) != g) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-__device__ __forceinline__ float ffn_gelu(float x) {
-  constexpr float kA = static_cast<float>(-2.0 * 0.7978845608028654);
-  constexpr float kB = static_cast<float>(0.044715);
-  const float x3 = __fmul_rn(__fmul_rn(x, x), x);
-  float z = __fmul_rn(kA, __fadd_rn(x, __fmul_rn(kB, x3)));
-  z = fminf(fmaxf(z, -87.0f), 88.0f);
-  return __fdiv_rn(x, __fadd_rn(1.0f, ffn_exp(z)));
+// gelu of the bf16 value with bits b (low 16 bits), for 2^-12 <= |y| < 16:
+// float64 evaluation (relative error below 2^-40; every such input's value
+// lies at least 1e-4 of a bf16 spacing from a rounding boundary) rounded once
+__device__ __noinline__ uint32_t gelu_bf16_exact(uint32_t b) {
+  const double y = static_cast<double>(__uint_as_float(b << 16));
+  const double u = 0.7978845608028654 * (y + 0.044715 * (y * y * y));
+  return f64_to_bf16_rn(y / (1.0 + exp(-2.0 * u)));
 }
 
-// The same two functions on a pair of values with the packed float32x2
-// operations (each lane of a packed op rounds exactly as the scalar op does,
-// so results are identical to ffn_exp / ffn_gelu element by element).
-__device__ __forceinline__ float2 ffn_exp_x2(float2 z) {
-  constexpr float kLog2e = static_cast<float>(1.4426950408889634);
-  constexpr float kLn2Hi = 0.693145751953125f;
-  constexpr float kLn2Lo = static_cast<float>(1.428606765330187e-06);
-  const float2 t = __fmul2_rn(z, make_float2(kLog2e, kLog2e));
-  const float2 n = make_float2(rintf(t.x), rintf(t.y));
-  const float2 r = __fadd2_rn(__fadd2_rn(z, __fmul2_rn(n, make_float2(-kLn2Hi, -kLn2Hi))),
-                              __fmul2_rn(n, make_float2(-kLn2Lo, -kLn2Lo)));
-  float2 p = make_float2(static_cast<float>(1.0 / 5040.0), static_cast<float>(1.0 / 5040.0));
-  const float c[7] = {static_cast<float>(1.0 / 720.0), static_cast<float>(1.0 / 120.0),
-                      static_cast<float>(1.0 / 24.0),  static_cast<float>(1.0 / 6.0),
-                      0.5f, 1.0f, 1.0f};
-#pragma unroll
-  for (int i = 0; i < 7; ++i) p = __fadd2_rn(__fmul2_rn(p, r), make_float2(c[i], c[i]));
-  const float2 scale = make_float2(__int_as_float((static_cast<int>(n.x) + 127) << 23),
-                                   __int_as_float((static_cast<int>(n.y) + 127) << 23));
-  return __fmul2_rn(p, scale);
+// the inputs outside the table (see above)
+__device__ __forceinline__ uint32_t gelu_bf16_outside(uint32_t b) {
+  const uint32_t mag = b & 0x7FFFu;
+  if (mag < kGeluTabBase) {
+    if (mag == 0u) return b;                                   // +-0
+    uint32_t f = __float_as_uint(__fmul_rn(__uint_as_float(b << 16), 0.5f));   // exact
+    f += (f >> 31) ? 0xFFFFFFFFu : 1u;                         // one float ulp toward +inf
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(f))));
+  }
+  if (mag > 0x7F80u || b == 0xFF80u) return 0x7FC0u;          // NaN, -inf
+  return (b & 0x8000u) ? 0x8000u : b;
 }
 
-__device__ __forceinline__ float2 ffn_gelu_x2(float2 x) {
-  constexpr float kA = static_cast<float>(-2.0 * 0.7978845608028654);
-  constexpr float kB = static_cast<float>(0.044715);
-  const float2 x3 = __fmul2_rn(__fmul2_rn(x, x), x);
-  float2 z = __fmul2_rn(make_float2(kA, kA), __fadd2_rn(x, __fmul2_rn(make_float2(kB, kB), x3)));
-  z.x = fminf(fmaxf(z.x, -87.0f), 88.0f);
-  z.y = fminf(fmaxf(z.y, -87.0f), 88.0f);
-  const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), ffn_exp_x2(z));
-  return make_float2(__fdiv_rn(x.x, d.x), __fdiv_rn(x.y, d.y));
+// entry i of the table: sign (i >> 11), offset (i & 2047) from 2^-12
+__device__ __forceinline__ void gelu_table_fill(uint16_t* tab, int tid, int nthreads) {
+  for (int i = tid; i < kGeluTabEntries; i += nthreads) {
+    const uint32_t b = (static_cast<uint32_t>(i & 0x800) << 4) | (kGeluTabBase + (i & 0x7FF));
+    tab[i] = static_cast<uint16_t>(gelu_bf16_exact(b));
+  }
+}
+
+// barrier `id` (1..15) over the first `nthreads` threads that reach it (a
+// multiple of 32; the other warps of the block do not take part)
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// table lookup for an input inside the table's range; `rel` = (b & 0x7FFF) -
+// kGeluTabBase (< 2048 there).  Outside the range the index wraps and the
+// caller must use gelu_bf16_outside instead.
+__device__ __forceinline__ uint32_t gelu_bf16_table(uint32_t tab, uint32_t b, uint32_t rel) {
+  return lds_u16(tab + 2u * ((rel & 0x7FFu) | ((b >> 4) & 0x800u)));
+}
+
+__device__ __forceinline__ uint32_t gelu_bf16(uint32_t tab, uint32_t b) {
+  const uint32_t rel = (b & 0x7FFFu) - kGeluTabBase;
+  return rel < 2048u ? gelu_bf16_table(tab, b, rel) : gelu_bf16_outside(b);
 }
 
 // ---------------------------------------------------------------------------

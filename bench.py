@@ -548,7 +548,7 @@ def run_reference(args):
 
 
 def run_ffn(args):
-    """The FFN pair at T=57600 (Wan2.2 block: 5120 -> 13824, GELU, 13824 -> 5120)
+    """The FFN pair at T=57600 ("ffn"; "ffn_mid": T=16384) (Wan2.2 block: 5120 -> 13824, GELU, 13824 -> 5120)
     with the down layer fed by the up layer's output.  Both layers are
     calibrated and packed before the timed region; a step is the online
     forward of one batch: fused (prep, up GEMM whose epilogue writes the down
@@ -565,6 +565,8 @@ def run_ffn(args):
     device = torch.device("cuda", local)
     active = dist_init("nccl", world, rank)
     Lu, Ld = synth.FULL_UP.with_(seed=1000 * rank), synth.FULL_DOWN
+    if args.workload == "ffn_mid":            # the same pair at T=16384 (profiling size)
+        Lu = synth.MID_UP.with_(seed=1000 * rank)
     T, d_model, d_ff = Lu.T, Lu.d_in, Lu.d_out
     X, W_up = synth.gen_layer(Lu, device)
     W_down = synth.gen_w(Ld.w, Ld.d_out, Ld.d_in, seed=Ld.seed + 1 + 1000 * rank, device=device)
@@ -644,7 +646,7 @@ def run_ffn(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
-            "config": {"workload": f"ffn: T={T} {d_model}->{d_ff} k={Lu.k} alpha={Lu.alpha}, GELU, "
+            "config": {"workload": f"{args.workload}: T={T} {d_model}->{d_ff} k={Lu.k} alpha={Lu.alpha}, GELU, "
                                    f"{d_ff}->{d_model} k={Ld.k} alpha={Ld.alpha}, "
                                    f"{LAYOUT_NAMES[Lu.layout]}",
                        "tokens_per_gpu": T, "parallelism": f"token shards x{world}",
@@ -679,7 +681,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="full",
                     choices=["full", "full_up", "full_down", "mid_up", "mid_down", "ffn0", "ffn2", "tiny",
-                             "sweep", "ffn"])
+                             "sweep", "ffn", "ffn_mid"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -687,7 +689,7 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)      # at least three untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "ffn":
+    elif args.workload in ("ffn", "ffn_mid"):
         run_ffn(args)
     else:
         run_gpu(args)

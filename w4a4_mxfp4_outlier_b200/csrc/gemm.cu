@@ -107,17 +107,20 @@ __device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], BfPai
 }
 
 // One lane's 32 columns col0 .. col0+31 of row `row` (as bf16 pairs) through
-// the fused FFN epilogue (see GemmArgs).  No warp collectives: callable per lane.
+// the fused FFN epilogue (see GemmArgs): writes the E2M1 codes of the MX
+// block they form and the outlier columns among them, and returns the
+// block's E8M0 scale code (0 where there is no block or no row), which the
+// caller stores 4 blocks at a time.  No warp collectives: callable per lane.
 // Not inlined: the epilogue calls it for 4 column chunks per tile, and with
 // four inlined copies the epilogue warps' code was large enough to push the
 // producer and MMA warps' instructions out of the instruction cache -- the
 // fused up-projection GEMM then ran at 0.49x the speed of this form
 // (T = 57600, 5120 -> 13824: 3.13 ms inlined, 1.87 ms called).
-__device__ __noinline__ void act_block(const BfPairs16 y, int row, int col0, const GemmArgs* ap,
-                                       uint32_t gelu_tab) {
+__device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0, const GemmArgs* ap,
+                                           uint32_t gelu_tab) {
   const uint32_t (&yb)[16] = y.w;
   const GemmArgs& a = *ap;
-  if (row >= a.T) return;
+  if (row >= a.T) return 0u;
   // bf16(gelu(y)) of the 32 columns as bf16 pairs: table lookups, with the
   // inputs outside the table's range (rare) redone afterwards
   uint32_t hp[16];
@@ -191,8 +194,17 @@ __device__ __noinline__ void act_block(const BfPairs16 y, int row, int col0, con
     }
     *reinterpret_cast<uint4*>(a.act_aq + static_cast<int64_t>(row) * a.act_nblk * 16 + b * 16) =
         make_uint4(w[0], w[1], w[2], w[3]);
-    a.act_sfa[sf_offset(row, b, a.act_nblk)] = static_cast<uint8_t>(code);
+    return code;
   }
+  return 0u;
+}
+
+// The scale codes of MX blocks b0 .. b0+3 of one row (b0 % 4 == 0): 4
+// contiguous bytes of the MMA layout, one word store.  act_nblk % 4 == 0, so
+// the 4 blocks are all J blocks or none is.
+__device__ __forceinline__ void act_store_scales(const GemmArgs& a, int row, int b0, uint32_t codes) {
+  if (b0 < a.act_nblk && row < a.T)
+    *reinterpret_cast<uint32_t*>(a.act_sfa + sf_offset(row, b0, a.act_nblk)) = codes;
 }
 
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
@@ -406,8 +418,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
       const int row = tm * BM + 32 * sp + lane;
       if constexpr (kAct) {
+        {
+          uint32_t codes = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * BN + 128 * half + 32 * c, &args, gelu_tab);
+          for (int c = 0; c < 4; ++c)
+            codes |= act_block(yb[c], row, tn * BN + 128 * half + 32 * c, &args, gelu_tab) << (8 * c);
+          act_store_scales(args, row, (tn * BN + 128 * half) >> 5, codes);
+        }
       } else if (row < args.T) {
         __nv_bfloat16* yrow = args.Y + static_cast<int64_t>(row) * args.ldy;
 #pragma unroll
@@ -729,8 +746,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
       if constexpr (kAct) {
         const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
+        uint32_t codes = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, &args, gelu_tab);
+        for (int c = 0; c < 4; ++c)
+          codes |= act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, &args, gelu_tab) << (8 * c);
+        act_store_scales(args, row, (tn * 256 + 128 * half) >> 5, codes);
         continue;
       }
       // Y through a per-warp staging block, 16 rows x 32 columns at a time:

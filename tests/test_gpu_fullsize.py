@@ -52,3 +52,44 @@ def test_full_size_sampled(L):
     Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
                                     ref_w["sfb"], ref_w["w_hp"])
     gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, L.name)
+
+
+def test_full_size_ffn_sampled():
+    """The fused FFN at T = 57600 as bench.py --workload ffn runs it (prep, up
+    GEMM with the GELU/prep epilogue, down GEMM): the down layer's codes,
+    scales and outlier columns on 1024 sampled rows against the oracle's prep
+    of bf16(gelu(Y_up)), Y_up from the library's plain up GEMM on those rows
+    (rows are independent and each output column accumulates in one fixed K
+    order, so it is the value the fused kernel rounded), and Y on those rows
+    within the product tolerance."""
+    from w4a4_mxfp4_outlier_b200 import ffn
+    Lu, Ld = synth.FULL_UP, synth.FULL_DOWN
+    X, W_up = gu.gen(Lu)
+    W_down = synth.gen_w(Ld.w, Ld.d_out, Ld.d_in, seed=Ld.seed + 1, device="cuda")
+    f = ffn.calibrate_ffn(X, W_up, W_down, Lu.alpha, Lu.k, Ld.alpha, Ld.k, Lu.layout)
+    Y = torch.empty((Lu.T, Lu.d_in), dtype=torch.bfloat16, device="cuda")
+    act_down = ffn.forward(X, f, Y)
+    st, bits = w4.last_error()
+    assert st == w4.OK, f"device error word {bits:#x}"
+
+    rows = synth.sample_rows(Lu.T, 1024).numpy()
+    ridx = torch.from_numpy(rows).cuda()
+    Xs = X[ridx].contiguous()
+    ws = torch.empty(w4.workspace_size(Xs.shape[0], Lu.d_in, Lu.d_out, Lu.k), dtype=torch.uint8,
+                     device="cuda")
+    Yu = torch.empty((Xs.shape[0], Lu.d_out), dtype=torch.bfloat16, device="cuda")
+    w4.linear(Xs, f.up_plain, ws, Yu)
+    Hn = orc.ffn_hidden(gu.to_np_f32(Yu))
+    c = gu.oracle_calib_from_gpu(f.down)
+    ref_a = orc.prep_activation(Hn, c["inv_s"], c["O"], c["J"])
+    d = f.down.dims
+    nb = ref_a["sfa"].shape[1]
+    np.testing.assert_array_equal(act_down.aq[ridx].cpu().numpy()[:, :nb * 16], ref_a["aq"])
+    sfa = gu.sf_canonical(act_down.sfa, rows, d.nblk, nb)
+    np.testing.assert_array_equal(sfa[:, :nb], ref_a["sfa"])
+    np.testing.assert_array_equal(gu.bf16_bits(act_down.xo[ridx])[:, :Ld.k], ref_a["xo"])
+
+    ref_w = orc.pack_weight(gu.to_np_f32(W_down), c["s"], c["O"], c["J"], Lu.layout)
+    Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
+                                    ref_w["sfb"], ref_w["w_hp"])
+    gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, "ffn_full_down")

@@ -23,7 +23,7 @@ ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["libw4a4.cu"]
-HEADERS = ["w4a4_device.cuh", "w4a4_internal.h", "w4a4_api.cu", "calib.cu", "prep.cu",
+HEADERS = ["w4a4_device.cuh", "w4a4_internal.h", "w4a4_api.cu", "calib.cu", "prep.cu", "prep_block.cu",
            "pack.cu", "gemm.cu", "noalloc.cu",
            "checkpoint.cu", "metrics.cu", "ffn.cu"]
 

@@ -5,6 +5,7 @@
 #include "calib.cu"
 #include "pack.cu"
 #include "prep.cu"
+#include "prep_block.cu"
 #include "gemm.cu"
 #include "noalloc.cu"
 #include "checkpoint.cu"

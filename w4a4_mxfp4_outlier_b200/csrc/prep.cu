@@ -7,6 +7,10 @@
 // sec. 3.2 ("at inference activations are first divided by s, then
 // quantised") and sec. 3.3 (X_J in 4 bits, X_O in high precision).
 //
+// Rows of at most 480 MX blocks (d_in up to 15360) go to the block-per-lane
+// form in prep_block.cu, which needs fewer instructions per element; this
+// kernel takes the wider rows (up to d_in = 16384).
+//
 // Design (HBM-bound in principle: 2 bytes read and ~0.56 bytes written per
 // element, so the instruction count per element is what has to stay low):
 //  * persistent grid, one CTA per SM; CTA b handles rows b, b+G, b+2G, ...
@@ -291,6 +295,8 @@ cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_
                         uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4,
                         const int32_t* rows) {
   if (T == 0) return cudaSuccess;
+  if (prep_block_supported(g))
+    return launch_prep_block(X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
   const PrepPlan p = plan_prep(g);
   const int sms = device_num_sms();
   const int grid = static_cast<int>(T < sms ? T : sms);

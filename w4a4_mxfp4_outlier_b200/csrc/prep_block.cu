@@ -1,0 +1,289 @@
+// Online activation preparation, block-per-lane form: the same computation as
+// prep_kernel (prep.cu) -- X times inv_s, outlier columns gathered to bf16,
+// the compacted remaining columns MXFP4-encoded into the MMA layout -- with
+// each consumer lane owning one whole 32-element MX block of the row.
+//
+// Method: paper review "W4A4 Quantization for Inference on Wan2.2-I2V-A14B",
+// sec. 3.2 (divide by s, then quantise) and sec. 3.3 (X_J in 4 bits, X_O in
+// high precision).
+//
+// Design (the kernel is issue-bound, so the point is fewer instructions per
+// element than prep_kernel's 8-elements-per-lane form):
+//  * the ring of rows in shared memory and its producer warp are those of
+//    prep_kernel (bulk copies of whole rows into kPrepStages fixed slots);
+//  * a group of `ntg` consumer threads handles one row, thread t the MX block
+//    t: its amax, scale and 16 code bytes need no shuffles (128x1 stripes
+//    take two, over the 4 lanes of a stripe);
+//  * `groups` groups (1, 2, 3 or 6) work on different ring slots, slot u
+//    belonging to group u % groups, so narrow rows still fill the SM;
+//  * each lane keeps the shared-memory offsets and inv_s of its 32 gathered
+//    elements in registers, in an order rotated by 2 * (lane / 2) elements:
+//    lanes of a warp then read 32 different banks although their blocks lie
+//    64 bytes apart; the 16 code bytes are rotated back before the store.
+#include "w4a4_internal.h"
+
+namespace w4a4 {
+
+// up to 480 consumers + the producer warp: 16 warps, 4 per scheduler, so each
+// thread may hold 128 registers (the 32 gather offsets and 32 inv_s of its
+// block, its 32 products, and the rest)
+constexpr int kPbMaxThreads = 512;
+
+// bf16 at byte offset `off` of the ring, widened to the bits of a float
+__device__ __forceinline__ float pb_ring_f32(const uint8_t* ring, uint32_t off) {
+  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(ring + off)) << 16);
+}
+
+__global__ void __launch_bounds__(kPbMaxThreads, 1)
+    prep_block_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t ldx, int d_in,
+                      const float* __restrict__ inv_s, const int32_t* __restrict__ O,
+                      const int32_t* __restrict__ jmap, int k, int k_pad, int kj, int nblk,
+                      int groups, int ntg, uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa,
+                      uint32_t* __restrict__ xo, int stripe4, const int32_t* __restrict__ rows) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kPrepStages) * kPrepStage);
+  uint64_t* empty = full + kPrepStages;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + kPrepStages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int u = 0; u < kPrepStages; ++u) {
+      mbar_init(&full[u], 1);
+      mbar_init(&empty[u], ntg / 32);
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  for (int u = threadIdx.x; u < kPrepStages; u += blockDim.x)
+    *reinterpret_cast<uint4*>(smem + static_cast<size_t>(u) * kPrepStage + kPrepZero) =
+        make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+
+  const int64_t nrows = T > blockIdx.x ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if (warp == 0) {
+    // ---------------- producer (whole warp; one elected lane issues) ----------------
+    const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
+    int64_t issued = 0;
+    int u = 0;
+    uint32_t ph = 0;
+    for (int64_t i = 0; i < nrows; ++i) {
+      if (i >= kPrepStages &&
+          !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
+        break;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&full[u], bytes);
+        const int64_t r = blockIdx.x + i * gridDim.x;
+        // output row r reads input row rows[r] when a row map is given
+        const uint16_t* from = X + (rows ? static_cast<int64_t>(rows[r]) : r) * ldx;
+        bulk_load(smem + static_cast<size_t>(u) * kPrepStage, from, bytes, &full[u]);
+      }
+      __syncwarp();
+      issued = i + 1;
+      if (++u == kPrepStages) {
+        u = 0;
+        ph ^= 1u;
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // do not leave bulk copies in flight into shared memory we give back
+      const int64_t first = issued > kPrepStages ? issued - kPrepStages : 0;
+      for (int64_t i = first; i < issued; ++i)
+        mbar_wait_bounded(&full[i % kPrepStages], static_cast<uint32_t>((i / kPrepStages) & 1),
+                          nullptr, DEVERR_TIMEOUT_PREP);
+    }
+    __syncwarp();
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int ct = threadIdx.x - 32;
+  const int g = ct / ntg;                   // group (uniform per warp: ntg % 32 == 0)
+  const int t = ct - g * ntg;               // MX block of the row this thread encodes
+  const bool enc = t < nblk;
+  const int m = lane >> 1;
+  const int rot = 2 * m;                    // processing order: element e reads (e + rot) mod 32
+  uint32_t go[32];
+  float2 isv[16];
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    uint32_t o0 = kPrepZero, o1 = kPrepZero;
+    float i0 = 1.f, i1 = 1.f;
+    const int p0 = 32 * t + ((e + rot) & 31);
+    const int p1 = 32 * t + ((e + 1 + rot) & 31);
+    if (enc && p0 < kj) {
+      const int j = jmap[p0];
+      o0 = 2u * static_cast<uint32_t>(j);
+      i0 = inv_s[j];
+    }
+    if (enc && p1 < kj) {
+      const int j = jmap[p1];
+      o1 = 2u * static_cast<uint32_t>(j);
+      i1 = inv_s[j];
+    }
+    go[e] = o0;
+    go[e + 1] = o1;
+    isv[e >> 1] = make_float2(i0, i1);
+  }
+  // the outlier pair this thread gathers on every row (more pairs than
+  // threads only when k > 2 * ntg; those run through the loop below)
+  const int xo_row = k_pad >> 1;                            // bf16 pairs per row of X_O
+  uint32_t oo0 = kPrepZero, oo1 = kPrepZero;
+  float2 oinv = make_float2(1.f, 1.f);
+  if (t < xo_row) {
+    const int o0 = 2 * t;
+    if (o0 < k) {
+      oo0 = 2u * static_cast<uint32_t>(O[o0]);
+      oinv.x = inv_s[O[o0]];
+    }
+    if (o0 + 1 < k) {
+      oo1 = 2u * static_cast<uint32_t>(O[o0 + 1]);
+      oinv.y = inv_s[O[o0 + 1]];
+    }
+  }
+  const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
+  const int64_t atoms_k = nblk >> 2;
+  const uint32_t ws = static_cast<uint32_t>(m) >> 2;        // the rotation back: whole words ...
+  const uint32_t bs = 8u * (static_cast<uint32_t>(m) & 3u);  // ... then bits
+  uint32_t ph = 0;
+  bool ok = true;
+
+  for (int64_t i0 = 0; i0 < nrows && ok; i0 += kPrepStages) {
+#pragma unroll
+    for (int u = 0; u < kPrepStages; ++u) {
+      if (u % groups != g) continue;
+      if (i0 + u >= nrows) break;
+      if (!warp_wait_bounded(&full[u], ph, abort_flag, DEVERR_TIMEOUT_PREP)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* ring = smem + u * kPrepStage;          // compile-time offset
+      const int64_t r = blockIdx.x + (i0 + u) * gridDim.x;
+      float2 v[16];
+      float amax = 0.f;
+      if (enc) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          v[e] = __fmul2_rn(make_float2(pb_ring_f32(ring, go[2 * e]), pb_ring_f32(ring, go[2 * e + 1])),
+                            isv[e]);
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          mx[e] = fmaxf(fmaxf(fabsf(v[2 * e].x), fabsf(v[2 * e].y)),
+                        fmaxf(fabsf(v[2 * e + 1].x), fabsf(v[2 * e + 1].y)));
+        amax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      }
+      if (stripe4) {                        // 128x1 stripes: the 4 lanes of 4 consecutive blocks
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      }
+      if (enc) {
+        const uint32_t code = mx_scale_code(amax);
+        const float inv = mx_inv_scale(code);
+        const float2 inv2 = make_float2(inv, inv);
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 a0 = __fmul2_rn(v[4 * q], inv2), a1 = __fmul2_rn(v[4 * q + 1], inv2);
+          const float2 a2 = __fmul2_rn(v[4 * q + 2], inv2), a3 = __fmul2_rn(v[4 * q + 3], inv2);
+          w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y);
+        }
+        // nibble e holds element (e + rot) mod 32: rotate the 128 bits left by
+        // 4 * rot = 32 * ws + bs bits
+        uint32_t a0 = w[0], a1 = w[1], a2 = w[2], a3 = w[3];
+        if (ws & 1u) {
+          const uint32_t tmp = a3;
+          a3 = a2;
+          a2 = a1;
+          a1 = a0;
+          a0 = tmp;
+        }
+        if (ws & 2u) {
+          uint32_t tmp = a0;
+          a0 = a2;
+          a2 = tmp;
+          tmp = a1;
+          a1 = a3;
+          a3 = tmp;
+        }
+        const uint4 out = make_uint4(__funnelshift_l(a3, a0, bs), __funnelshift_l(a0, a1, bs),
+                                     __funnelshift_l(a1, a2, bs), __funnelshift_l(a2, a3, bs));
+        *reinterpret_cast<uint4*>(aq + r * aq_row + 16 * t) = out;
+        const int64_t sf_row = (((r >> 7) * atoms_k) << 9) + ((r & 31) << 4) + (((r & 127) >> 5) << 2);
+        sfa[sf_row + ((t >> 2) << 9) + (t & 3)] = static_cast<uint8_t>(code);
+      }
+      if (t < xo_row) {
+        uint32_t* xo_p = xo + r * xo_row;
+        const float x0 = pb_ring_f32(ring, oo0);
+        const float x1 = pb_ring_f32(ring, oo1);
+        const float2 vv = __fmul2_rn(make_float2(x0, x1), oinv);
+        xo_p[t] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(vv.x))) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(vv.y))) << 16);
+        for (int i2 = t + ntg; i2 < xo_row; i2 += ntg) {
+          const int o0 = 2 * i2;
+          const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : kPrepZero;
+          const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : kPrepZero;
+          const float y0 = __fmul_rn(pb_ring_f32(ring, a0), o0 < k ? inv_s[O[o0]] : 1.f);
+          const float y1 = __fmul_rn(pb_ring_f32(ring, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
+          xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
+                     (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[u]);
+    }
+    ph ^= 1u;
+  }
+}
+
+struct PrepBlockPlan {
+  int groups, ntg;
+};
+
+// Threads per group: one per MX block (and at least one per outlier pair up
+// to 512), rounded to warps; groups: the most of 6, 3, 2, 1 (divisors of the
+// ring's slot count) that fit the thread limit.  ntg == 0: not supported.
+static PrepBlockPlan plan_prep_block(const Geometry& g) {
+  const int nblk = static_cast<int>(g.nblk);
+  const int xo_pairs = static_cast<int>(g.k_pad / 2);
+  int need = nblk > 0 ? nblk : 1;
+  if (xo_pairs > need) need = xo_pairs < kPbMaxThreads - 32 ? xo_pairs : kPbMaxThreads - 32;
+  const int ntg = static_cast<int>(round_up(need, 32));
+  if (nblk > kPbMaxThreads - 32) return {0, 0};
+  const int cand[4] = {6, 3, 2, 1};
+  for (int c : cand)
+    if (c * ntg + 32 <= kPbMaxThreads) return {c, ntg};
+  return {0, 0};
+}
+
+static constexpr size_t kPrepBlockSmem =
+    static_cast<size_t>(kPrepStages) * kPrepStage + 2 * kPrepStages * 8 + 16;
+
+bool prep_block_supported(const Geometry& g) {
+  return g.d_in <= kPrepMaxD && plan_prep_block(g).ntg > 0;
+}
+
+cudaError_t launch_prep_block(const void* X, int64_t T, int64_t ldx, const float* inv_s,
+                              const int32_t* O, const int32_t* jmap, const Geometry& g,
+                              uint8_t* aq, uint8_t* sfa, void* xo, cudaStream_t stream,
+                              bool stripe4, const int32_t* rows) {
+  if (T == 0) return cudaSuccess;
+  const PrepBlockPlan p = plan_prep_block(g);
+  if (p.ntg == 0) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(prep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kPrepBlockSmem));
+  if (e != cudaSuccess) return e;
+  const int sms = device_num_sms();
+  const int grid = static_cast<int>(T < sms ? T : sms);
+  prep_block_kernel<<<grid, p.groups * p.ntg + 32, kPrepBlockSmem, stream>>>(
+      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
+      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
+      static_cast<int>(g.nblk), p.groups, p.ntg, aq, sfa, static_cast<uint32_t*>(xo),
+      stripe4 ? 1 : 0, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace w4a4

@@ -61,6 +61,12 @@ cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_
                         uint8_t* sfa, void* xo, cudaStream_t stream, bool stripe4 = false,
                         const int32_t* rows = nullptr);
 bool prep_supported(const Geometry& g);
+// The block-per-lane form of the same computation (prep_block.cu).
+bool prep_block_supported(const Geometry& g);
+cudaError_t launch_prep_block(const void* X, int64_t T, int64_t ldx, const float* inv_s,
+                              const int32_t* O, const int32_t* jmap, const Geometry& g,
+                              uint8_t* aq, uint8_t* sfa, void* xo, cudaStream_t stream,
+                              bool stripe4, const int32_t* rows);
 // Outputs of the fused FFN epilogue: the next layer's activation buffers
 // (Aq, SFA, X_O) and its inv_s in this layer's output-column order.
 struct ActOut {

@@ -40,10 +40,13 @@ constexpr int kPrepMaxD = 16384;
 // consumer threads per CTA for CH chunks each, and the register cap that
 // lets that many (+ the producer warp) run in one CTA: the state kept per
 // chunk is 8 offsets + 8 inv_s registers
+// (the warps of a block are spread over the SM's 4 schedulers, each with a
+// quarter of the register file: ceil(warps / 4) * 32 * registers <= 16384)
 template <int CH> struct PrepCfg;
 template <> struct PrepCfg<1> { static constexpr int kMaxConsumers = 992, kMaxRegs = 64; };
 template <> struct PrepCfg<2> { static constexpr int kMaxConsumers = 736, kMaxRegs = 80; };
-template <> struct PrepCfg<4> { static constexpr int kMaxConsumers = 512, kMaxRegs = 120; };
+template <> struct PrepCfg<4> { static constexpr int kMaxConsumers = 480, kMaxRegs = 128; };
+template <> struct PrepCfg<8> { static constexpr int kMaxConsumers = 256, kMaxRegs = 168; };
 
 // bf16 at byte offset `off` of the ring, widened to the bits of a float
 __device__ __forceinline__ uint32_t ring_bf16(const uint8_t* ring, uint32_t off) {
@@ -258,6 +261,7 @@ static PrepPlan plan_prep(const Geometry& g) {
   PrepPlan p{1, 0};
   if (nchunks > PrepCfg<1>::kMaxConsumers) p.ch = 2;
   if (nchunks > 2 * PrepCfg<2>::kMaxConsumers) p.ch = 4;
+  if (nchunks > 4 * PrepCfg<4>::kMaxConsumers) p.ch = 8;
   int nt = (nchunks + p.ch - 1) / p.ch;
   nt = static_cast<int>(round_up(nt < 32 ? 32 : nt, 32));
   p.nt = nt;
@@ -270,7 +274,7 @@ static constexpr size_t kPrepSmem =
 bool prep_supported(const Geometry& g) {
   if (g.d_in > kPrepMaxD) return false;
   const int nchunks = static_cast<int>(g.kj_pad / 8);
-  return nchunks <= 4 * PrepCfg<4>::kMaxConsumers;
+  return nchunks <= 8 * PrepCfg<8>::kMaxConsumers;
 }
 
 template <int CH>
@@ -303,13 +307,19 @@ cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_
   switch (p.ch) {
     case 1: return launch_prep_ch<1>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
     case 2: return launch_prep_ch<2>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
-    default: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 4: return launch_prep_ch<4>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    default: return launch_prep_ch<8>(p, grid, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
   }
 }
 
 
-static_assert((PrepCfg<1>::kMaxConsumers + 32) * PrepCfg<1>::kMaxRegs <= 65536, "CH=1 registers");
-static_assert((PrepCfg<2>::kMaxConsumers + 32) * PrepCfg<2>::kMaxRegs <= 65536, "CH=2 registers");
-static_assert((PrepCfg<4>::kMaxConsumers + 32) * PrepCfg<4>::kMaxRegs <= 65536, "CH=4 registers");
+template <int CH>
+constexpr bool prep_regs_fit() {
+  return ((PrepCfg<CH>::kMaxConsumers + 32) / 32 + 3) / 4 * 32 * PrepCfg<CH>::kMaxRegs <= 16384;
+}
+static_assert(prep_regs_fit<1>(), "CH=1 registers");
+static_assert(prep_regs_fit<2>(), "CH=2 registers");
+static_assert(prep_regs_fit<4>(), "CH=4 registers");
+static_assert(prep_regs_fit<8>(), "CH=8 registers");
 
 }  // namespace w4a4

@@ -27,12 +27,25 @@ __global__ void __launch_bounds__(256) colabsmax_kernel(const uint16_t* __restri
     const int64_t rstep = static_cast<int64_t>(gridDim.y) * 8;
     int64_t r = static_cast<int64_t>(blockIdx.y) * 8 + threadIdx.y;
     const uint16_t* p = A + col0;
-    // four rows in flight per iteration
-    for (; r + 3 * rstep < rows; r += 4 * rstep) {
+    // eight rows in flight per iteration, folded pairwise (measured against
+    // four: 5.98 -> 6.61 TB/s on a 57600 x 5120 X)
+    for (; r + 7 * rstep < rows; r += 8 * rstep) {
+      uint4 u0 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 4 * rstep) * lda));
+      uint4 u1 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 5 * rstep) * lda));
+      uint4 u2 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 6 * rstep) * lda));
+      uint4 u3 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 7 * rstep) * lda));
       uint4 v0 = __ldcs(reinterpret_cast<const uint4*>(p + r * lda));
       uint4 v1 = __ldcs(reinterpret_cast<const uint4*>(p + (r + rstep) * lda));
       uint4 v2 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 2 * rstep) * lda));
       uint4 v3 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 3 * rstep) * lda));
+      v0.x = __vmaxu2(v0.x & 0x7FFF7FFFu, u0.x & 0x7FFF7FFFu); v0.y = __vmaxu2(v0.y & 0x7FFF7FFFu, u0.y & 0x7FFF7FFFu);
+      v0.z = __vmaxu2(v0.z & 0x7FFF7FFFu, u0.z & 0x7FFF7FFFu); v0.w = __vmaxu2(v0.w & 0x7FFF7FFFu, u0.w & 0x7FFF7FFFu);
+      v1.x = __vmaxu2(v1.x & 0x7FFF7FFFu, u1.x & 0x7FFF7FFFu); v1.y = __vmaxu2(v1.y & 0x7FFF7FFFu, u1.y & 0x7FFF7FFFu);
+      v1.z = __vmaxu2(v1.z & 0x7FFF7FFFu, u1.z & 0x7FFF7FFFu); v1.w = __vmaxu2(v1.w & 0x7FFF7FFFu, u1.w & 0x7FFF7FFFu);
+      v2.x = __vmaxu2(v2.x & 0x7FFF7FFFu, u2.x & 0x7FFF7FFFu); v2.y = __vmaxu2(v2.y & 0x7FFF7FFFu, u2.y & 0x7FFF7FFFu);
+      v2.z = __vmaxu2(v2.z & 0x7FFF7FFFu, u2.z & 0x7FFF7FFFu); v2.w = __vmaxu2(v2.w & 0x7FFF7FFFu, u2.w & 0x7FFF7FFFu);
+      v3.x = __vmaxu2(v3.x & 0x7FFF7FFFu, u3.x & 0x7FFF7FFFu); v3.y = __vmaxu2(v3.y & 0x7FFF7FFFu, u3.y & 0x7FFF7FFFu);
+      v3.z = __vmaxu2(v3.z & 0x7FFF7FFFu, u3.z & 0x7FFF7FFFu); v3.w = __vmaxu2(v3.w & 0x7FFF7FFFu, u3.w & 0x7FFF7FFFu);
       m[0] = __vmaxu2(m[0], __vmaxu2(__vmaxu2(v0.x & 0x7FFF7FFFu, v1.x & 0x7FFF7FFFu),
                                      __vmaxu2(v2.x & 0x7FFF7FFFu, v3.x & 0x7FFF7FFFu)));
       m[1] = __vmaxu2(m[1], __vmaxu2(__vmaxu2(v0.y & 0x7FFF7FFFu, v1.y & 0x7FFF7FFFu),

@@ -186,9 +186,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "6aa35026cdb7bf54ff41c662e438cd1c225aaabc42485e0d472f50a59bf3554f",
+    "sha256": "3207cd2ba8bf63c553cce1799e84b192489c022c068e5f075229f0d67a2f790e",
     "workload": "full",
-    "bytes_per_launch": (750766336 + 1558680832 + 1657089536 + 572224256) / 2,
+    "bytes_per_launch": (718466048 + 1563207680 + 1352207104 + 573537536) / 2,
 }
 
 

@@ -95,6 +95,91 @@ def aggregate(per_rank_units: float, world: int, step_s_max: float) -> float:
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons read through NVML every 5 ms in a
+    background thread (the same counters nvidia-smi prints; reading them
+    changes nothing).  Only samples inside the timed window are summarised."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_power_brake_slowdown", 0x80),
+               ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, handle, nvml):
+        self.h = handle
+        self.nvml = nvml
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.window = (None, None)
+        self.max_mhz = None
+
+    @staticmethod
+    def open(local_index: int):
+        """An NVML sampler for CUDA device `local_index`, or None."""
+        try:
+            import pynvml as nvml
+            import torch
+            nvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(local_index)
+            bus = getattr(prop, "pci_bus_id", None)
+            if bus is not None:
+                busid = "%08X:%02X:%02X.0" % (getattr(prop, "pci_domain_id", 0), bus,
+                                              getattr(prop, "pci_device_id", 0))
+                h = nvml.nvmlDeviceGetHandleByPciBusId(busid)
+            else:
+                h = nvml.nvmlDeviceGetHandleByIndex(local_index)
+            nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM)
+            return NvmlClockSampler(h, nvml)
+        except Exception:
+            return None
+
+    def start(self):
+        try:
+            self.max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+        except Exception:
+            self.max_mhz = None
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        n = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append((time.time(), float(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)),
+                                     n.nvmlDeviceGetPowerUsage(self.h) / 1000.0,
+                                     int(n.nvmlDeviceGetCurrentClocksEventReasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def mark_start(self):
+        self.window = (time.time(), None)
+
+    def mark_end(self):
+        self.window = (self.window[0], time.time())
+
+    def stop(self):
+        self.stop_evt.set()
+        if self.thread:
+            self.thread.join(timeout=2)
+        t0, t1 = self.window
+        inside = [x for x in self.samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": ["no samples in the timed window"], "samples_total": len(self.samples),
+                    "source": "nvml, 5 ms"}
+        reasons = sorted({name for _, _, _, r in inside for name, bit in self.REASONS if r & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside),
+                "sm_min_mhz": min(x[1] for x in inside),
+                "sm_max_mhz": self.max_mhz if self.max_mhz else max(x[1] for x in inside),
+                "power_w_max": max(x[2] for x in inside), "samples": len(inside),
+                "reasons": reasons, "source": "nvml, 5 ms"}
+
+
+def clock_sampler(local_index: int):
+    """NVML sampling where it works, nvidia-smi otherwise."""
+    s = NvmlClockSampler.open(local_index)
+    return s if s is not None else ClockSampler(local_index)
+
+
 class ClockSampler:
     """nvidia-smi samples every 20 ms; only samples whose timestamp falls inside
     the timed window are summarised."""
@@ -204,6 +289,16 @@ def gemm_traffic(workload: str):
     return int(GEMM_TRAFFIC["bytes_per_launch"])
 
 
+def peak_keys(timed_seconds: float):
+    """(peak used, the other one): the burst bf16 figure for a timed region
+    shorter than a second of back-to-back work (the measured burst figure is
+    the best of ten sub-millisecond GEMMs), the sustained one (measured over a
+    4 s loop under the power cap) for longer regions."""
+    if timed_seconds >= 1.0:
+        return "bf16_tflops_sustained", "bf16_tflops"
+    return "bf16_tflops", "bf16_tflops_sustained"
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -294,7 +389,7 @@ def run_gpu(args):
     mk = lambda: torch.cuda.Event(enable_timing=True)
     evs = [[{"off": [mk(), mk()], "on": [mk(), mk(), mk()]} for _ in runs] for _ in range(args.steps)]
     t0, t1 = mk(), mk()
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     torch.cuda.synchronize()
     dist_barrier(active, device)
     clocks.start()
@@ -332,12 +427,9 @@ def run_gpu(args):
     online_tflops = flops / ((sum(gemm_ms) + sum(prep_ms)) * 1e-3) / 1e12
 
     peaks, src = measured_peaks()
-    # burst figure when the timed window ran at full clock, sustained one when the power cap bit
-    boost = (clock_info.get("sm_mhz") and clock_info.get("sm_max_mhz")
-             and clock_info["sm_mhz"] >= 0.95 * clock_info["sm_max_mhz"])
-    key = "bf16_tflops" if boost else "bf16_tflops_sustained"
+    key, other_key = peak_keys(step_ms * args.steps * 1e-3)
     fp4_peak = peaks[key] * FP4_PER_BF16
-    other = peaks["bf16_tflops_sustained" if boost else "bf16_tflops"] * FP4_PER_BF16
+    other = peaks[other_key] * FP4_PER_BF16
     roof = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
             "traffic": gemm_traffic(args.workload),
@@ -606,7 +698,7 @@ def run_ffn(args):
 
     evs = [[mk() for _ in range(4)] for _ in range(args.steps)]
     t0, t1, u0, u1 = mk(), mk(), mk(), mk()
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     torch.cuda.synchronize()
     dist_barrier(active, device)
     clocks.start()
@@ -635,9 +727,7 @@ def run_ffn(args):
     prep_ms, up_ms, down_ms = avg(0, 1), avg(1, 2), avg(2, 3)
     gemm_tflops = flops / ((up_ms + down_ms) * 1e-3) / 1e12
     peaks, src = measured_peaks()
-    boost = (clock_info.get("sm_mhz") and clock_info.get("sm_max_mhz")
-             and clock_info["sm_mhz"] >= 0.95 * clock_info["sm_max_mhz"])
-    key = "bf16_tflops" if boost else "bf16_tflops_sustained"
+    key, _ = peak_keys(step_ms * args.steps * 1e-3)
     fp4_peak = peaks[key] * FP4_PER_BF16
     if rank == 0:
         out = {

@@ -75,3 +75,62 @@ def test_reference_arm_prints_on_rank0_only(monkeypatch):
 
 
 
+
+
+def test_peak_choice_by_timed_region_length():
+    assert bench.peak_keys(0.04) == ("bf16_tflops", "bf16_tflops_sustained")
+    assert bench.peak_keys(1.5) == ("bf16_tflops_sustained", "bf16_tflops")
+
+
+class _FakeNvml:
+    """Stands in for pynvml: the clock drops under a power cap from `switch`
+    (a time.time() value) on."""
+    NVML_CLOCK_SM = 0
+
+    def __init__(self):
+        self.switch = float("inf")
+
+    def _capped(self):
+        import time
+        return time.time() >= self.switch
+
+    def nvmlDeviceGetMaxClockInfo(self, h, which):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        return 1400 if self._capped() else 1965
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 1000000 if self._capped() else 600000        # milliwatts
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 if self._capped() else 0x0               # sw_power_cap
+
+
+def test_nvml_sampler_summarises_the_timed_window():
+    import time
+    fake = _FakeNvml()
+    s = bench.NvmlClockSampler(object(), fake)
+    s.start()
+    time.sleep(0.03)
+    fake.switch = time.time()
+    s.mark_start()
+    time.sleep(0.12)
+    s.mark_end()
+    fake.switch = float("inf")
+    time.sleep(0.03)
+    out = s.stop()
+    assert out["source"] == "nvml, 5 ms" and out["samples"] >= 3
+    assert out["sm_max_mhz"] == 1965.0 and out["sm_mhz"] == 1400.0 and out["sm_min_mhz"] == 1400.0
+    assert out["reasons"] == ["sw_power_cap"] and out["power_w_max"] == 1000.0
+    # samples outside the window are not counted
+    assert out["samples"] < len(s.samples)
+
+
+def test_clock_sampler_without_nvml_or_nvidia_smi():
+    s = bench.clock_sampler(0)          # no GPU here: NVML fails, nvidia-smi is absent
+    s.start()
+    s.mark_start()
+    s.mark_end()
+    out = s.stop()
+    assert out["sm_mhz"] is None and out["reasons"]

@@ -93,3 +93,47 @@ def test_full_size_ffn_sampled():
     Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
                                     ref_w["sfb"], ref_w["w_hp"])
     gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, "ffn_full_down")
+
+
+SWEEP_EXTREMES = [L for L in synth.sweep_layers()
+                  if (L.k, L.layout, L.alpha) in ((0, 1, 0.5), (256, 1, 0.5), (16, 2, 0.7), (256, 2, 0.7))]
+
+
+@pytest.mark.parametrize("L", SWEEP_EXTREMES, ids=lambda L: L.name)
+def test_sweep_sampled(L):
+    """Sweep points at their own size (T = 16384, 5120 -> 13824) with the
+    32x32-tile and 128x1-stripe weight scales and the smallest and largest k:
+    the packed weight in full, codes and Y on 512 sampled token rows."""
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
+    act = w4.alloc_act(L.T, pw)
+    Y = torch.empty((L.T, L.d_out), dtype=torch.bfloat16, device="cuda")
+    w4.prep_act(X, pw, act)
+    w4.gemm_dual(act, L.T, pw, Y)
+    st, bits = w4.last_error()
+    assert st == w4.OK, f"device error word {bits:#x}"
+    c = gu.oracle_calib_from_gpu(pw)
+    np.testing.assert_array_equal(pw.O.cpu().numpy(), c["O"])
+    ref_w = orc.pack_weight(gu.to_np_f32(W), c["s"], c["O"], c["J"], L.layout)
+    d = pw.dims
+    nb = ref_w["sfb"].shape[1]
+    np.testing.assert_array_equal(pw.wq.view(L.d_out, -1).cpu().numpy()[:, :nb * 16], ref_w["wq"])
+    if d.nblk:
+        sfb = gu.sf_canonical(pw.sfb, d.sfb_rows, d.nblk, nb)
+        np.testing.assert_array_equal(sfb[:L.d_out, :nb], ref_w["sfb"])
+    if L.k:
+        np.testing.assert_array_equal(gu.bf16_bits(pw.w_hp).reshape(L.d_out, d.k_pad)[:, :L.k],
+                                      ref_w["w_hp"])
+
+    rows = synth.sample_rows(L.T, 512).numpy()
+    ridx = torch.from_numpy(rows).cuda()
+    ref_a = orc.prep_activation(gu.to_np_f32(X[ridx]), c["inv_s"], c["O"], c["J"])
+    np.testing.assert_array_equal(act.aq[ridx].cpu().numpy()[:, :nb * 16], ref_a["aq"])
+    if d.nblk:
+        sfa = gu.sf_canonical(act.sfa, rows, d.nblk, nb)
+        np.testing.assert_array_equal(sfa[:, :nb], ref_a["sfa"])
+    if L.k:
+        np.testing.assert_array_equal(gu.bf16_bits(act.xo[ridx])[:, :L.k], ref_a["xo"])
+    Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
+                                    ref_w["sfb"], ref_w["w_hp"])
+    gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, L.name)

@@ -117,7 +117,7 @@ __device__ __forceinline__ void pack_bf16_pairs(const uint32_t (&acc)[32], BfPai
 // fused up-projection GEMM then ran at 0.49x the speed of this form
 // (T = 57600, 5120 -> 13824: 3.13 ms inlined, 1.87 ms called).
 __device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0, const GemmArgs* ap,
-                                           uint32_t gelu_tab) {
+                                           uint32_t gelu_tab, uint32_t stg) {
   const uint32_t (&yb)[16] = y.w;
   const GemmArgs& a = *ap;
   if (row >= a.T) return 0u;
@@ -192,8 +192,16 @@ __device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0,
       const float2 a2 = __fmul2_rn(v[4 * q + 2], inv2), a3 = __fmul2_rn(v[4 * q + 3], inv2);
       w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y);
     }
-    *reinterpret_cast<uint4*>(a.act_aq + static_cast<int64_t>(row) * a.act_nblk * 16 + b * 16) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+    if (stg != 0u) {
+      // the staging row of this lane: 16-byte chunk (b & 3) at the 64-byte
+      // swizzle position the tile store expects
+      const uint32_t lane = threadIdx.x & 31u;
+      st_shared_v4(stg + 64u * lane + 16u * ((static_cast<uint32_t>(b) & 3u) ^ ((lane >> 1) & 3u)),
+                   w[0], w[1], w[2], w[3]);
+    } else {
+      *reinterpret_cast<uint4*>(a.act_aq + static_cast<int64_t>(row) * a.act_nblk * 16 + b * 16) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
     return code;
   }
   return 0u;
@@ -422,7 +430,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint32_t codes = 0;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            codes |= act_block(yb[c], row, tn * BN + 128 * half + 32 * c, &args, gelu_tab) << (8 * c);
+            codes |= act_block(yb[c], row, tn * BN + 128 * half + 32 * c, &args, gelu_tab, 0u) << (8 * c);
           act_store_scales(args, row, (tn * BN + 128 * half) >> 5, codes);
         }
       } else if (row < args.T) {
@@ -483,13 +491,18 @@ constexpr int P_EPI_ARRIVALS = 2 * NUM_EPI_WARPS;
 
 constexpr int P_EPI_BYTES = 16 * 64;          // staging block: 16 rows x 32 bf16 (64-byte swizzle)
 
+// The plain kernel: 6 stages, a 1 KB Y staging block per epilogue warp.  The
+// fused FFN kernel: 5 stages, a 2 KB block per warp (its 32 rows x 64 code
+// bytes of one tile half) and the GELU table.
+template <bool kAct>
 struct PairSmem {
-  uint8_t stage[P_STAGES][P_STAGE_BYTES];
-  // per epilogue warp: Y staging; the fused FFN epilogue (no Y) keeps its
-  // GELU table here instead
-  alignas(1024) uint8_t epi[NUM_EPI_WARPS][P_EPI_BYTES];
-  uint64_t full[P_STAGES];     // leader's counts the bytes of both CTAs
-  uint64_t empty[P_STAGES];    // both CTAs: MMA commit, multicast
+  static constexpr int kStages = kAct ? 5 : P_STAGES;
+  static constexpr int kEpiBytes = kAct ? 32 * 64 : P_EPI_BYTES;
+  uint8_t stage[kStages][P_STAGE_BYTES];
+  alignas(1024) uint8_t epi[NUM_EPI_WARPS][kEpiBytes];
+  alignas(16) uint16_t gelu_tab[kAct ? kGeluTabEntries : 8];
+  uint64_t full[kStages];      // leader's counts the bytes of both CTAs
+  uint64_t empty[kStages];     // both CTAs: MMA commit, multicast
   uint64_t acc_full;           // both CTAs: MMA commit, multicast
   uint64_t acc_empty;          // leader: epilogue warps of both CTAs
   uint64_t drain;
@@ -504,7 +517,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                           const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ GemmArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  PairSmem& sm = *reinterpret_cast<PairSmem*>(
+  using Smem = PairSmem<kAct>;
+  constexpr int NST = Smem::kStages;
+  Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   volatile uint32_t* abort_flag = &sm.abort_flag;
 
@@ -517,7 +532,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int nkt = args.kt_o + args.kt_j;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < P_STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int m_rows = tm * 256 + 128 * static_cast<int>(rank);
       const int n_rows = tn * 256 + 128 * static_cast<int>(rank);
       for (int kt = 0; kt < nkt; ++kt, ++it) {
-        if (it >= P_STAGES &&
+        if (it >= NST &&
             !warp_wait_bounded(&sm.empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
           ok = false;
           break;
@@ -590,7 +605,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         __syncwarp();
         issued = it + 1;
-        if (++s == P_STAGES) {
+        if (++s == NST) {
           s = 0;
           ph ^= 1u;
         }
@@ -600,9 +615,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (rank == 0) {
         // wait for the stages posted in the last ring's worth of K tiles, so
         // no copy lands after teardown (earlier ones were consumed)
-        const uint32_t first = issued > P_STAGES ? issued - P_STAGES : 0;
+        const uint32_t first = issued > NST ? issued - NST : 0;
         for (uint32_t i = first; i < issued; ++i)
-          mbar_wait_bounded(&sm.full[i % P_STAGES], (i / P_STAGES) & 1u, nullptr,
+          mbar_wait_bounded(&sm.full[i % NST], (i / NST) & 1u, nullptr,
                             DEVERR_TIMEOUT_PRODUCER);
       }
       spin_ns(50000);            // the peer CTA's copies land on the leader's barriers
@@ -653,7 +668,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           __syncwarp();
           acc = 1;
-          if (++s == P_STAGES) {
+          if (++s == NST) {
             s = 0;
             ph ^= 1u;
             soff = 0;
@@ -687,7 +702,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           __syncwarp();
           acc = 1;
           buf ^= TMEM_SF_BUF;
-          if (++s == P_STAGES) {
+          if (++s == NST) {
             s = 0;
             ph ^= 1u;
             soff = 0;
@@ -714,11 +729,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&sm.acc_empty), 0);
     uint32_t gelu_tab = 0;
     if constexpr (kAct) {
-      static_assert(sizeof(sm.epi) >= kGeluTabEntries * sizeof(uint16_t), "GELU table space");
-      uint16_t* tab = reinterpret_cast<uint16_t*>(&sm.epi[0][0]);
-      gelu_table_fill(tab, ew * 32 + lane, NUM_EPI_WARPS * 32);
+      gelu_table_fill(sm.gelu_tab, ew * 32 + lane, NUM_EPI_WARPS * 32);
       named_bar_sync(1, NUM_EPI_WARPS * 32);
-      gelu_tab = smem_u32(tab);
+      gelu_tab = smem_u32(sm.gelu_tab);
     }
     uint32_t tcount = 0;
     for (int t = pair; t < ntiles; t += npairs, ++tcount) {
@@ -745,12 +758,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
       if constexpr (kAct) {
-        const int row = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp + lane;
+        // the codes of 4 consecutive MX blocks b0 .. b0+3 (64 bytes per row)
+        // go through this warp's staging block, 32 rows x 64 bytes, and leave
+        // in one TMA tile store (tm_y maps act_aq here; rows past T clipped)
+        const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp;
+        const int row = row0 + lane;
+        const int b0 = (tn * 256 + 128 * half) >> 5;
+        const uint32_t stg = smem_u32(sm.epi[ew]);
+        if (elect_one()) bulk_wait_group_read0();   // the previous tile's store has read it
+        __syncwarp();
         uint32_t codes = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          codes |= act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, &args, gelu_tab) << (8 * c);
-        act_store_scales(args, row, (tn * 256 + 128 * half) >> 5, codes);
+          codes |= act_block(yb[c], row, tn * 256 + 128 * half + 32 * c, &args, gelu_tab, stg) << (8 * c);
+        act_store_scales(args, row, b0, codes);
+        if (b0 < args.act_nblk) {                   // uniform over the warp
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (elect_one()) {
+            tma_store_2d(&tm_y, stg, b0 * 16, row0);
+            bulk_commit_group();
+          }
+          __syncwarp();
+        }
         continue;
       }
       // Y through a per-warp staging block, 16 rows x 32 columns at a time:
@@ -849,7 +879,8 @@ static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 }
 
 size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
-size_t gemm_pair_smem_bytes() { return sizeof(PairSmem) + 1024; }
+template <bool kAct>
+size_t gemm_pair_smem_bytes() { return sizeof(PairSmem<kAct>) + 1024; }
 
 // Number of co-resident CTA pairs of the pair kernel on this device (0 if the
 // query fails); cached per device.
@@ -858,11 +889,12 @@ static int pair_capacity() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] > 0) return cached[dev];
-  const size_t smem = gemm_pair_smem_bytes();
+  const size_t smem = gemm_pair_smem_bytes<false>();
+  const size_t smem_act = gemm_pair_smem_bytes<true>();
   if (cudaFuncSetAttribute(gemm_dual_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess ||
       cudaFuncSetAttribute(gemm_dual_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+                           static_cast<int>(smem_act)) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 148, 1, 1);
@@ -877,8 +909,10 @@ static int pair_capacity() {
   cfg.numAttrs = 1;
   int n = 0;
   int n2 = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel<false>, &cfg) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n2, gemm_dual_pair_kernel<true>, &cfg) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel<false>, &cfg) != cudaSuccess)
+    return 0;
+  cfg.dynamicSmemBytes = smem_act;
+  if (cudaOccupancyMaxActiveClusters(&n2, gemm_dual_pair_kernel<true>, &cfg) != cudaSuccess ||
       n <= 0 || n2 <= 0)
     return 0;
   if (n2 < n) n = n2;
@@ -948,7 +982,7 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   const int ntiles = a.tiles_m * a.tiles_n;
   if (pair) {
     const int npairs = ntiles < pair_capacity() ? ntiles : pair_capacity();
-    const size_t smem = gemm_pair_smem_bytes();
+    const size_t smem = act ? gemm_pair_smem_bytes<true>() : gemm_pair_smem_bytes<false>();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * npairs, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
@@ -964,9 +998,16 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
     // Y as bf16 tiles of 16 rows x 32 columns, 64-byte swizzle (epilogue staging layout)
     CUtensorMap tm_y;
     memset(&tm_y, 0, sizeof(tm_y));
-    if (act != nullptr)
+    if (act != nullptr) {
+      // the next layer's codes as tiles of 32 rows x 64 bytes, 64-byte swizzle
+      if (act->nblk > 0 &&
+          !make_tmap(&tm_y, act->aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                     static_cast<uint64_t>(act->nblk) * 16, T, static_cast<uint64_t>(act->nblk) * 16,
+                     32, 64, false, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
       return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true>, tm_a, tm_b, tm_ao, tm_bo,
                                 tm_sfa, tm_sfb, tm_y, a);
+    }
     if (!make_tmap(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
                    static_cast<uint64_t>(ldy) * 2, 16, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;

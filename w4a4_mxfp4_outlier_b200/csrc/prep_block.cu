@@ -14,8 +14,13 @@
 //  * a group of `ntg` consumer threads handles one row, thread t the MX block
 //    t: its amax, scale and 16 code bytes need no shuffles (128x1 stripes
 //    take two, over the 4 lanes of a stripe);
-//  * `groups` groups (1, 2, 3 or 6) work on different ring slots, slot u
-//    belonging to group u % groups, so narrow rows still fill the SM;
+//  * G = 6 / S groups (1, 2, 3 or 6) work on different ring slots, group g
+//    owning the S consecutive slots g*S .. g*S + S - 1, so narrow rows still
+//    fill the SM.  The group's slot base is folded into its lanes' gather
+//    offsets and the loop over its S slots is unrolled, so every group runs
+//    the same S copies of the loop body with the slot offset as the loads'
+//    immediate (owning every G-th slot instead made the groups run different
+//    copies and stall on instruction fetch);
 //  * each lane keeps the shared-memory offsets and inv_s of its 32 gathered
 //    elements in registers, in an order rotated by 2 * (lane / 2) elements:
 //    lanes of a warp then read 32 different banks although their blocks lie
@@ -34,11 +39,12 @@ __device__ __forceinline__ float pb_ring_f32(const uint8_t* ring, uint32_t off) 
   return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(ring + off)) << 16);
 }
 
+template <int S>
 __global__ void __launch_bounds__(kPbMaxThreads, 1)
     prep_block_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t ldx, int d_in,
                       const float* __restrict__ inv_s, const int32_t* __restrict__ O,
                       const int32_t* __restrict__ jmap, int k, int k_pad, int kj, int nblk,
-                      int groups, int ntg, uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa,
+                      int ntg, uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa,
                       uint32_t* __restrict__ xo, int stripe4, const int32_t* __restrict__ rows) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kPrepStages) * kPrepStage);
@@ -105,6 +111,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   const bool enc = t < nblk;
   const int m = lane >> 1;
   const int rot = 2 * m;                    // processing order: element e reads (e + rot) mod 32
+  const uint32_t gbase = static_cast<uint32_t>(g * S * kPrepStage);   // this group's first slot
   uint32_t go[32];
   float2 isv[16];
 #pragma unroll
@@ -123,8 +130,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
       o1 = 2u * static_cast<uint32_t>(j);
       i1 = inv_s[j];
     }
-    go[e] = o0;
-    go[e + 1] = o1;
+    go[e] = gbase + o0;
+    go[e + 1] = gbase + o1;
     isv[e >> 1] = make_float2(i0, i1);
   }
   // the outlier pair this thread gathers on every row (more pairs than
@@ -150,16 +157,20 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   uint32_t ph = 0;
   bool ok = true;
 
+  oo0 += gbase;
+  oo1 += gbase;
+
   for (int64_t i0 = 0; i0 < nrows && ok; i0 += kPrepStages) {
 #pragma unroll
-    for (int u = 0; u < kPrepStages; ++u) {
-      if (u % groups != g) continue;
+    for (int j = 0; j < S; ++j) {
+      const int u = g * S + j;
       if (i0 + u >= nrows) break;
       if (!warp_wait_bounded(&full[u], ph, abort_flag, DEVERR_TIMEOUT_PREP)) {
         ok = false;
         break;
       }
-      const uint8_t* ring = smem + u * kPrepStage;          // compile-time offset
+      const uint8_t* ring = smem + j * kPrepStage;          // compile-time offset (+ gbase in go)
+      const uint8_t* slot = ring + gbase;
       const int64_t r = blockIdx.x + (i0 + u) * gridDim.x;
       float2 v[16];
       float amax = 0.f;
@@ -226,8 +237,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
           const int o0 = 2 * i2;
           const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : kPrepZero;
           const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : kPrepZero;
-          const float y0 = __fmul_rn(pb_ring_f32(ring, a0), o0 < k ? inv_s[O[o0]] : 1.f);
-          const float y1 = __fmul_rn(pb_ring_f32(ring, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
+          const float y0 = __fmul_rn(pb_ring_f32(slot, a0), o0 < k ? inv_s[O[o0]] : 1.f);
+          const float y1 = __fmul_rn(pb_ring_f32(slot, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
           xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
                      (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
         }
@@ -262,6 +273,24 @@ static PrepBlockPlan plan_prep_block(const Geometry& g) {
 static constexpr size_t kPrepBlockSmem =
     static_cast<size_t>(kPrepStages) * kPrepStage + 2 * kPrepStages * 8 + 16;
 
+template <int S>
+static cudaError_t launch_prep_block_s(const PrepBlockPlan& p, const void* X, int64_t T, int64_t ldx,
+                                       const float* inv_s, const int32_t* O, const int32_t* jmap,
+                                       const Geometry& g, uint8_t* aq, uint8_t* sfa, void* xo,
+                                       cudaStream_t stream, bool stripe4, const int32_t* rows) {
+  static_assert(kPrepStages % S == 0, "groups own whole blocks of ring slots");
+  cudaError_t e = cudaFuncSetAttribute(prep_block_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kPrepBlockSmem));
+  if (e != cudaSuccess) return e;
+  const int sms = device_num_sms();
+  const int grid = static_cast<int>(T < sms ? T : sms);
+  prep_block_kernel<S><<<grid, p.groups * p.ntg + 32, kPrepBlockSmem, stream>>>(
+      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
+      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
+      static_cast<int>(g.nblk), p.ntg, aq, sfa, static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
+  return cudaGetLastError();
+}
+
 bool prep_block_supported(const Geometry& g) {
   return g.d_in <= kPrepMaxD && plan_prep_block(g).ntg > 0;
 }
@@ -273,17 +302,12 @@ cudaError_t launch_prep_block(const void* X, int64_t T, int64_t ldx, const float
   if (T == 0) return cudaSuccess;
   const PrepBlockPlan p = plan_prep_block(g);
   if (p.ntg == 0) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(prep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kPrepBlockSmem));
-  if (e != cudaSuccess) return e;
-  const int sms = device_num_sms();
-  const int grid = static_cast<int>(T < sms ? T : sms);
-  prep_block_kernel<<<grid, p.groups * p.ntg + 32, kPrepBlockSmem, stream>>>(
-      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
-      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
-      static_cast<int>(g.nblk), p.groups, p.ntg, aq, sfa, static_cast<uint32_t*>(xo),
-      stripe4 ? 1 : 0, rows);
-  return cudaGetLastError();
+  switch (p.groups) {
+    case 1: return launch_prep_block_s<6>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 2: return launch_prep_block_s<3>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 3: return launch_prep_block_s<2>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    default: return launch_prep_block_s<1>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+  }
 }
 
 }  // namespace w4a4

@@ -40,17 +40,20 @@ MID128 = MID.with_(name="mid_k64_128x1", layout=2, k=64)
 SMALL = [TINY, RAGGED, RAGGED32, RAGGED128, K0, KFULL, T1, SINGLE]
 
 # the prep kernel's launch shapes: block-per-lane form with 2 thread groups
-# (192 blocks), with 1 group at its 480-block limit, with more outlier pairs
+# (192 blocks; with the 6-slot ring at d_in 6144 and the 18-slot ring for
+# short rows at 5440; 6 and 3 groups on short rows are the small shapes and
+# FFN0), with 1 group at its 480-block limit, with more outlier pairs
 # than blocks (k = 900) and more than its 480 lanes (k = 1500: the extra pairs
 # loop); the 8-columns-per-lane form past 480 blocks (d_in = 16384, also with
 # 128x1 stripes)
 G2 = synth.Layer("prep_g2_d6144", 200, 6144, 272, 0.6, 20, 0, synth.X_UP, synth.W_UP)
+G2N = synth.Layer("prep_g2_d5440", 230, 5440, 256, 0.6, 20, 0, synth.X_UP, synth.W_UP)
 B480 = synth.Layer("prep_b480_d15360", 150, 15360, 256, 0.6, 16, 0, synth.X_UP, synth.W_UP)
 XOWIDE = synth.Layer("prep_xo_k900", 160, 1024, 256, 0.5, 900, 0, synth.X_UP, synth.W_UP)
 XOLOOP = synth.Layer("prep_xo_k1500", 100, 2048, 256, 0.5, 1500, 0, synth.X_UP, synth.W_UP)
 WIDE = synth.Layer("prep_wide_d16384", 300, 16384, 256, 0.6, 40, 0, synth.X_UP, synth.W_UP)
 WIDE128 = WIDE.with_(name="prep_wide_d16384_128x1", layout=2, k=24)
-PREP_SHAPES = [G2, B480, XOWIDE, XOLOOP, WIDE, WIDE128]
+PREP_SHAPES = [G2, G2N, B480, XOWIDE, XOLOOP, WIDE, WIDE128]
 
 
 def _calibrate(L):

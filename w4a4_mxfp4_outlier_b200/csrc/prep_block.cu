@@ -9,12 +9,13 @@
 //
 // Design (the kernel is issue-bound, so the point is fewer instructions per
 // element than prep_kernel's 8-elements-per-lane form):
-//  * the ring of rows in shared memory and its producer warp are those of
-//    prep_kernel (bulk copies of whole rows into kPrepStages fixed slots);
+//  * a ring of rows in shared memory filled by a producer warp with bulk
+//    copies of whole rows, as in prep_kernel (its 6 slots of 32.9 KB, or 18
+//    slots of 11 KB for rows of up to 5480 elements);
 //  * a group of `ntg` consumer threads handles one row, thread t the MX block
 //    t: its amax, scale and 16 code bytes need no shuffles (128x1 stripes
 //    take two, over the 4 lanes of a stripe);
-//  * G = 6 / S groups (1, 2, 3 or 6) work on different ring slots, group g
+//  * G = slots / S groups (1, 2, 3 or 6) work on different ring slots, group g
 //    owning the S consecutive slots g*S .. g*S + S - 1, so narrow rows still
 //    fill the SM.  The group's slot base is folded into its lanes' gather
 //    offsets and the loop over its S slots is unrolled, so every group runs
@@ -34,12 +35,24 @@ namespace w4a4 {
 // block, its 32 products, and the rest)
 constexpr int kPbMaxThreads = 512;
 
+// The ring: NSLOT slots of SLOT bytes, a row plus a 16-byte zero slot each.
+// Wide rows use prep_kernel's 6 x 32.9 KB; rows of up to 5480 elements use
+// 18 x 11 KB (the same shared memory), so three times as many rows are in
+// flight where a row is short.
+template <int NSLOT, int SLOT>
+struct PbRing {
+  static constexpr int kSlots = NSLOT, kSlot = SLOT, kZero = SLOT - 16;
+  static constexpr size_t kSmem = static_cast<size_t>(NSLOT) * SLOT + 2 * NSLOT * 8 + 16;
+};
+using PbWide = PbRing<kPrepStages, kPrepStage>;
+using PbNarrow = PbRing<18, 10976>;
+
 // bf16 at byte offset `off` of the ring, widened to the bits of a float
 __device__ __forceinline__ float pb_ring_f32(const uint8_t* ring, uint32_t off) {
   return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(ring + off)) << 16);
 }
 
-template <int S>
+template <int S, class R>
 __global__ void __launch_bounds__(kPbMaxThreads, 1)
     prep_block_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t ldx, int d_in,
                       const float* __restrict__ inv_s, const int32_t* __restrict__ O,
@@ -47,23 +60,23 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
                       int ntg, uint8_t* __restrict__ aq, uint8_t* __restrict__ sfa,
                       uint32_t* __restrict__ xo, int stripe4, const int32_t* __restrict__ rows) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kPrepStages) * kPrepStage);
-  uint64_t* empty = full + kPrepStages;
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + kPrepStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(R::kSlots) * R::kSlot);
+  uint64_t* empty = full + R::kSlots;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + R::kSlots);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int u = 0; u < kPrepStages; ++u) {
+    for (int u = 0; u < R::kSlots; ++u) {
       mbar_init(&full[u], 1);
       mbar_init(&empty[u], ntg / 32);
     }
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  for (int u = threadIdx.x; u < kPrepStages; u += blockDim.x)
-    *reinterpret_cast<uint4*>(smem + static_cast<size_t>(u) * kPrepStage + kPrepZero) =
+  for (int u = threadIdx.x; u < R::kSlots; u += blockDim.x)
+    *reinterpret_cast<uint4*>(smem + static_cast<size_t>(u) * R::kSlot + R::kZero) =
         make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
@@ -76,7 +89,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
     int u = 0;
     uint32_t ph = 0;
     for (int64_t i = 0; i < nrows; ++i) {
-      if (i >= kPrepStages &&
+      if (i >= R::kSlots &&
           !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
         break;
       if (elect_one()) {
@@ -84,20 +97,20 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         const int64_t r = blockIdx.x + i * gridDim.x;
         // output row r reads input row rows[r] when a row map is given
         const uint16_t* from = X + (rows ? static_cast<int64_t>(rows[r]) : r) * ldx;
-        bulk_load(smem + static_cast<size_t>(u) * kPrepStage, from, bytes, &full[u]);
+        bulk_load(smem + static_cast<size_t>(u) * R::kSlot, from, bytes, &full[u]);
       }
       __syncwarp();
       issued = i + 1;
-      if (++u == kPrepStages) {
+      if (++u == R::kSlots) {
         u = 0;
         ph ^= 1u;
       }
     }
     if (lane == 0 && *abort_flag) {
       // do not leave bulk copies in flight into shared memory we give back
-      const int64_t first = issued > kPrepStages ? issued - kPrepStages : 0;
+      const int64_t first = issued > R::kSlots ? issued - R::kSlots : 0;
       for (int64_t i = first; i < issued; ++i)
-        mbar_wait_bounded(&full[i % kPrepStages], static_cast<uint32_t>((i / kPrepStages) & 1),
+        mbar_wait_bounded(&full[i % R::kSlots], static_cast<uint32_t>((i / R::kSlots) & 1),
                           nullptr, DEVERR_TIMEOUT_PREP);
     }
     __syncwarp();
@@ -111,12 +124,12 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   const bool enc = t < nblk;
   const int m = lane >> 1;
   const int rot = 2 * m;                    // processing order: element e reads (e + rot) mod 32
-  const uint32_t gbase = static_cast<uint32_t>(g * S * kPrepStage);   // this group's first slot
+  const uint32_t gbase = static_cast<uint32_t>(g * S * R::kSlot);   // this group's first slot
   uint32_t go[32];
   float2 isv[16];
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    uint32_t o0 = kPrepZero, o1 = kPrepZero;
+    uint32_t o0 = R::kZero, o1 = R::kZero;
     float i0 = 1.f, i1 = 1.f;
     const int p0 = 32 * t + ((e + rot) & 31);
     const int p1 = 32 * t + ((e + 1 + rot) & 31);
@@ -137,7 +150,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   // the outlier pair this thread gathers on every row (more pairs than
   // threads only when k > 2 * ntg; those run through the loop below)
   const int xo_row = k_pad >> 1;                            // bf16 pairs per row of X_O
-  uint32_t oo0 = kPrepZero, oo1 = kPrepZero;
+  uint32_t oo0 = R::kZero, oo1 = R::kZero;
   float2 oinv = make_float2(1.f, 1.f);
   if (t < xo_row) {
     const int o0 = 2 * t;
@@ -160,7 +173,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   oo0 += gbase;
   oo1 += gbase;
 
-  for (int64_t i0 = 0; i0 < nrows && ok; i0 += kPrepStages) {
+  for (int64_t i0 = 0; i0 < nrows && ok; i0 += R::kSlots) {
 #pragma unroll
     for (int j = 0; j < S; ++j) {
       const int u = g * S + j;
@@ -169,7 +182,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         ok = false;
         break;
       }
-      const uint8_t* ring = smem + j * kPrepStage;          // compile-time offset (+ gbase in go)
+      const uint8_t* ring = smem + j * R::kSlot;          // compile-time offset (+ gbase in go)
       const uint8_t* slot = ring + gbase;
       const int64_t r = blockIdx.x + (i0 + u) * gridDim.x;
       float2 v[16];
@@ -235,8 +248,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(vv.y))) << 16);
         for (int i2 = t + ntg; i2 < xo_row; i2 += ntg) {
           const int o0 = 2 * i2;
-          const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : kPrepZero;
-          const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : kPrepZero;
+          const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : R::kZero;
+          const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : R::kZero;
           const float y0 = __fmul_rn(pb_ring_f32(slot, a0), o0 < k ? inv_s[O[o0]] : 1.f);
           const float y1 = __fmul_rn(pb_ring_f32(slot, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
           xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
@@ -270,21 +283,19 @@ static PrepBlockPlan plan_prep_block(const Geometry& g) {
   return {0, 0};
 }
 
-static constexpr size_t kPrepBlockSmem =
-    static_cast<size_t>(kPrepStages) * kPrepStage + 2 * kPrepStages * 8 + 16;
-
-template <int S>
+template <int S, class R>
 static cudaError_t launch_prep_block_s(const PrepBlockPlan& p, const void* X, int64_t T, int64_t ldx,
                                        const float* inv_s, const int32_t* O, const int32_t* jmap,
                                        const Geometry& g, uint8_t* aq, uint8_t* sfa, void* xo,
                                        cudaStream_t stream, bool stripe4, const int32_t* rows) {
-  static_assert(kPrepStages % S == 0, "groups own whole blocks of ring slots");
-  cudaError_t e = cudaFuncSetAttribute(prep_block_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kPrepBlockSmem));
+  static_assert(R::kSlots % S == 0, "groups own whole blocks of ring slots");
+  cudaError_t e = cudaFuncSetAttribute(prep_block_kernel<S, R>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(R::kSmem));
   if (e != cudaSuccess) return e;
   const int sms = device_num_sms();
   const int grid = static_cast<int>(T < sms ? T : sms);
-  prep_block_kernel<S><<<grid, p.groups * p.ntg + 32, kPrepBlockSmem, stream>>>(
+  prep_block_kernel<S, R><<<grid, p.groups * p.ntg + 32, R::kSmem, stream>>>(
       static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
       static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
       static_cast<int>(g.nblk), p.ntg, aq, sfa, static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
@@ -302,11 +313,20 @@ cudaError_t launch_prep_block(const void* X, int64_t T, int64_t ldx, const float
   if (T == 0) return cudaSuccess;
   const PrepBlockPlan p = plan_prep_block(g);
   if (p.ntg == 0) return cudaErrorInvalidValue;
+  // short rows: the 18-slot ring unless a single group would have to unroll
+  // all 18 slots
+  if (2 * g.d_in + 16 <= PbNarrow::kSlot && p.groups > 1) {
+    switch (p.groups) {
+      case 2: return launch_prep_block_s<9, PbNarrow>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+      case 3: return launch_prep_block_s<6, PbNarrow>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+      default: return launch_prep_block_s<3, PbNarrow>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    }
+  }
   switch (p.groups) {
-    case 1: return launch_prep_block_s<6>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
-    case 2: return launch_prep_block_s<3>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
-    case 3: return launch_prep_block_s<2>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
-    default: return launch_prep_block_s<1>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 1: return launch_prep_block_s<6, PbWide>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 2: return launch_prep_block_s<3, PbWide>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    case 3: return launch_prep_block_s<2, PbWide>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
+    default: return launch_prep_block_s<1, PbWide>(p, X, T, ldx, inv_s, O, jmap, g, aq, sfa, xo, stream, stripe4, rows);
   }
 }
 

@@ -271,9 +271,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "3207cd2ba8bf63c553cce1799e84b192489c022c068e5f075229f0d67a2f790e",
+    "sha256": "bdc61dd4ac7910c5bbbdb2ee73ec00021bf52707ab3cb1b013b449de54c91425",
     "workload": "full",
-    "bytes_per_launch": (718466048 + 1563207680 + 1352207104 + 573537536) / 2,
+    "bytes_per_launch": (723234560 + 1563205888 + 1461546240 + 573794048) / 2,
 }
 
 

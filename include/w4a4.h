@@ -243,7 +243,8 @@ w4a4_status w4a4_packed_load(const void* host, size_t bytes, const w4a4_packed_w
  * whether fused or not.  +inf maps to +inf, -inf and NaN to NaN.
  *
  * Fused use: calibrate and pack the down layer, w4a4_ffn_link it, pack the up
- * weight with w4a4_pack_weight_rows(rows = perm), then per batch
+ * weight in its natural channel order and reorder that pack with
+ * w4a4_permute_packed_rows(rows = perm), then per batch
  * w4a4_prep_act (up) -> w4a4_gemm_dual_act (up, writing the down layer's Aq,
  * SFA, X_O) -> w4a4_gemm_dual (down).
  * ------------------------------------------------------------------------ */
@@ -263,9 +264,23 @@ w4a4_status w4a4_ffn_link(const w4a4_packed_weight* next, int32_t* perm, float* 
                           void* stream);
 
 /* w4a4_pack_weight with the rows of W permuted: packed output channel n is
- * W row rows[n] (rows: int32 [d_out] device array). */
+ * W row rows[n] (rows: int32 [d_out] device array).  This packs the permuted
+ * matrix: with 32x32 tiles, a tile groups 32 consecutive permuted rows, so
+ * the result differs from a reordered natural pack; for the fused FFN use
+ * w4a4_permute_packed_rows. */
 w4a4_status w4a4_pack_weight_rows(const void* W, int64_t ldw, const float* s, const int32_t* rows,
                                   const w4a4_packed_weight* pw, void* stream);
+
+/* dst = src with its output channels reordered: packed row r of dst is packed
+ * row rows[r] of src (rows: int32 [d_out] device array, a permutation) -- the
+ * E2M1 codes, the E8M0 scales (each row keeps its scale from src, so 32x32
+ * tiles stay the tiles of src's channel order) and the bf16 outlier rows.
+ * src and dst: same d_in, d_out, k and layout, distinct buffers; dst's
+ * input-side arrays (s, inv_s, O, jmap) are not written (the caller shares
+ * or copies them).  Asynchronous on `stream`.  Errors: INVALID_ARG for
+ * mismatched shapes, a null `rows` or shared output buffers. */
+w4a4_status w4a4_permute_packed_rows(const w4a4_packed_weight* src, const int32_t* rows,
+                                     const w4a4_packed_weight* dst, void* stream);
 
 /* The up projection with the fused FFN epilogue: computes the dual-branch
  * product of (aq, sfa, xo) with pw (packed with rows = perm) and, instead of

@@ -56,11 +56,38 @@ def test_pack_rows_matches_permuted_pack(layout):
     np.testing.assert_array_equal(gu.bf16_bits(pr.w_hp).reshape(L.d_out, -1)[:, :L.k], ref["w_hp"])
 
 
+@pytest.mark.parametrize("layout", [0, 1, 2])
+def test_permute_packed_rows_matches_reordered_natural_pack(layout):
+    L = synth.Layer("perm", 64, 512, 368, 0.6, 9, layout, XS, synth.WSpec(0.02), seed=4)
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, layout)
+    perm = torch.from_numpy(np.random.default_rng(1).permutation(L.d_out).astype(np.int32)).cuda()
+    pr = w4.alloc_packed(L.d_in, L.d_out, L.k, layout)
+    pr.s, pr.inv_s, pr.O, pr.jmap = pw.s, pw.inv_s, pw.O, pw.jmap
+    import ctypes
+    st = w4._permute_packed_rows(ctypes.byref(pw.c), perm.data_ptr(), ctypes.byref(pr.c), None)
+    assert st == w4.OK
+    torch.cuda.synchronize()
+    c = gu.oracle_calib_from_gpu(pw)
+    ref = orc.pack_weight(gu.to_np_f32(W), c["s"], c["O"], c["J"], layout)
+    p = perm.cpu().numpy()
+    nb = ref["sfb"].shape[1]
+    np.testing.assert_array_equal(pr.wq.view(L.d_out, -1).cpu().numpy()[:, :nb * 16], ref["wq"][p])
+    d = pr.dims
+    sfb = gu.sf_canonical(pr.sfb, d.sfb_rows, d.nblk, nb)
+    np.testing.assert_array_equal(sfb[:L.d_out, :nb], ref["sfb"][p])
+    np.testing.assert_array_equal(gu.bf16_bits(pr.w_hp).reshape(L.d_out, -1)[:, :L.k], ref["w_hp"][p])
+    # in place is refused
+    assert w4._permute_packed_rows(ctypes.byref(pw.c), perm.data_ptr(), ctypes.byref(pw.c),
+                                   None) == w4.ERR_INVALID_ARG
+
+
 FFN_CASES = [
     # T, d_model, d_ff, k_up, k_down, layout
     (300, 512, 1376, 8, 19, 0),      # pair GEMM; ragged d_ff; kj_pad of the down layer > d_ff
     (100, 256, 640, 4, 32, 2),       # single-CTA GEMM (T <= 128), 128x1 stripes
     (520, 1024, 2048, 16, 0, 1),     # no outliers in the down layer, 32x32 tiles
+    (300, 512, 1376, 8, 19, 1),      # 32x32 tiles with a non-trivial channel order
 ]
 
 

@@ -1,0 +1,115 @@
+"""Seeded random shapes through the whole path (calibration, packing, prep,
+GEMM) against the oracle: T from 1 to 700 (single-CTA and pair GEMM, ragged
+tiles), d_in from 8 to 6000 in steps of 8, d_out from 16 to 1200 in steps of
+16, k from 0 to d_in, all three weight-scale layouts and a spread of alpha.
+The codes, scales, outlier columns and packed weight bit for bit; Y within
+the product tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import w4a4_mxfp4_outlier_b200 as w4
+from w4a4_mxfp4_outlier_b200 import ffn
+from oracle import w4a4_oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def _cases(n=40, seed=2024):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        T = int(rng.choice([1, 7, 64, 128, 129, 255, 300, 513, 700]))
+        d_in = int(rng.integers(1, 751)) * 8
+        d_out = int(rng.integers(1, 76)) * 16
+        k = int(rng.choice([0, 1, 3, 16, 33, d_in // 7, d_in]))
+        k = min(k, d_in)
+        layout = int(rng.integers(0, 3))
+        alpha = float(rng.choice([0.3, 0.5, 0.6, 0.8]))
+        planted = int(min(d_in, rng.integers(0, 24)))
+        xs = synth.XSpec("student3", 0.3, planted, 8.0, 30.0)
+        out.append(synth.Layer(f"rand{i}_T{T}_{d_in}x{d_out}_k{k}_l{layout}", T, d_in, d_out, alpha,
+                               k, layout, xs, synth.WSpec(0.02), seed=100 + i))
+    return out
+
+
+@pytest.mark.parametrize("L", _cases(), ids=lambda L: L.name)
+def test_random_shape_parity(L):
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
+    act = w4.alloc_act(L.T, pw)
+    w4.prep_act(X, pw, act)
+    Y = torch.empty((L.T, L.d_out), dtype=torch.bfloat16, device="cuda")
+    w4.gemm_dual(act, L.T, pw, Y)
+    torch.cuda.synchronize()
+    st, bits = w4.last_error()
+    assert st == w4.OK, hex(bits)
+
+    c = gu.oracle_calib_from_gpu(pw)
+    np.testing.assert_array_equal(pw.O.cpu().numpy(), c["O"])
+    Xn, Wn = gu.to_np_f32(X), gu.to_np_f32(W)
+    ref_w = orc.pack_weight(Wn, c["s"], c["O"], c["J"], L.layout)
+    ref_a = orc.prep_activation(Xn, c["inv_s"], c["O"], c["J"])
+    d = pw.dims
+    nb = ref_a["sfa"].shape[1]
+    np.testing.assert_array_equal(pw.wq.view(L.d_out, -1).cpu().numpy()[:, :nb * 16], ref_w["wq"])
+    np.testing.assert_array_equal(act.aq.cpu().numpy()[:, :nb * 16], ref_a["aq"])
+    if d.nblk:
+        np.testing.assert_array_equal(gu.sf_canonical(pw.sfb, d.sfb_rows, d.nblk, nb)[:L.d_out, :nb],
+                                      ref_w["sfb"])
+        np.testing.assert_array_equal(gu.sf_canonical(act.sfa, L.T, d.nblk, nb)[:, :nb], ref_a["sfa"])
+    if L.k:
+        np.testing.assert_array_equal(gu.bf16_bits(act.xo)[:, :L.k], ref_a["xo"])
+        np.testing.assert_array_equal(gu.bf16_bits(pw.w_hp).reshape(L.d_out, d.k_pad)[:, :L.k],
+                                      ref_w["w_hp"])
+    Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
+                                    ref_w["sfb"], ref_w["w_hp"])
+    gu.check_tolerance(gu.to_np_f32(Y).astype(np.float64), Y_ref, L.name)
+
+
+def _ffn_cases(n=8, seed=77):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        T = int(rng.choice([5, 128, 200, 333, 600]))
+        d_model = int(rng.integers(2, 97)) * 16
+        d_ff = int(rng.integers(2, 161)) * 16
+        k_up = int(min(d_model, rng.choice([0, 4, 16, 40])))
+        k_down = int(min(d_ff, rng.choice([0, 7, 19, 64, d_ff])))
+        layout = int(rng.integers(0, 3))
+        out.append((f"ffn{i}_T{T}_{d_model}x{d_ff}_k{k_up}_{k_down}_l{layout}", T, d_model, d_ff,
+                    k_up, k_down, layout, 100 + i))
+    return out
+
+
+@pytest.mark.parametrize("case", _ffn_cases(), ids=lambda c: c[0])
+def test_random_ffn_parity(case):
+    _, T, d_model, d_ff, k_up, k_down, layout, seed = case
+    xs = synth.XSpec("student3", 0.3, min(d_model, 6), 8.0, 30.0)
+    Lx = synth.Layer("rffn", T, d_model, d_ff, 0.6, k_up, layout, xs, synth.WSpec(0.02), seed=seed)
+    X, W_up = gu.gen(Lx)
+    W_down = synth.gen_w(synth.WSpec(0.015), d_model, d_ff, seed=seed + 50, device="cuda")
+    f = ffn.calibrate_ffn(X, W_up, W_down, 0.6, k_up, 0.7, k_down, layout)
+    Y_f = torch.empty((T, d_model), dtype=torch.bfloat16, device="cuda")
+    act_down = ffn.forward(X, f, Y_f)
+    Y_u = torch.empty_like(Y_f)
+    ffn.forward_unfused(X, f, Y_u)
+    torch.cuda.synchronize()
+    st, bits = w4.last_error()
+    assert st == w4.OK, hex(bits)
+    assert torch.equal(Y_f.view(torch.int16), Y_u.view(torch.int16))
+    # the fused epilogue's codes against the oracle's prep of bf16(gelu(Y_up))
+    ws = torch.empty(w4.workspace_size(T, d_model, d_ff, k_up), dtype=torch.uint8, device="cuda")
+    Yu = torch.empty((T, d_ff), dtype=torch.bfloat16, device="cuda")
+    w4.linear(X, f.up_plain, ws, Yu)
+    c = gu.oracle_calib_from_gpu(f.down)
+    ref = orc.prep_activation(orc.ffn_hidden(gu.to_np_f32(Yu)), c["inv_s"], c["O"], c["J"])
+    d = f.down.dims
+    nb = ref["sfa"].shape[1]
+    np.testing.assert_array_equal(act_down.aq.cpu().numpy()[:, :nb * 16], ref["aq"])
+    if d.nblk:
+        np.testing.assert_array_equal(gu.sf_canonical(act_down.sfa, T, d.nblk, nb)[:, :nb], ref["sfa"])
+    if k_down:
+        np.testing.assert_array_equal(gu.bf16_bits(act_down.xo)[:, :k_down], ref["xo"])

@@ -89,6 +89,8 @@ _gelu_bf16 = _sig("w4a4_gelu_bf16", _st, _vp, _i64, _i64, _i64, _vp, _i64, _vp)
 _ffn_link = _sig("w4a4_ffn_link", _st, ctypes.POINTER(PackedWeightC), _vp, _vp, _vp)
 _pack_weight_rows = _sig("w4a4_pack_weight_rows", _st, _vp, _i64, _vp, _vp,
                          ctypes.POINTER(PackedWeightC), _vp)
+_permute_packed_rows = _sig("w4a4_permute_packed_rows", _st, ctypes.POINTER(PackedWeightC), _vp,
+                            ctypes.POINTER(PackedWeightC), _vp)
 _gemm_dual_act = _sig("w4a4_gemm_dual_act", _st, _vp, _vp, _vp, _i64, ctypes.POINTER(PackedWeightC),
                       ctypes.POINTER(PackedWeightC), _vp, _vp, _vp, _vp, _vp)
 _error_sums = _sig("w4a4_error_sums", _st, _vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp)
@@ -100,7 +102,7 @@ EXPORTED = [
     "w4a4_workspace_size", "w4a4_prep_act", "w4a4_gemm_dual", "w4a4_linear",
     "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
     "w4a4_packed_image_size", "w4a4_packed_save", "w4a4_packed_image_info", "w4a4_packed_load",
-    "w4a4_error_sums", "w4a4_gelu_bf16", "w4a4_ffn_link", "w4a4_pack_weight_rows",
+    "w4a4_error_sums", "w4a4_gelu_bf16", "w4a4_ffn_link", "w4a4_pack_weight_rows", "w4a4_permute_packed_rows",
     "w4a4_gemm_dual_act",
 ]
 

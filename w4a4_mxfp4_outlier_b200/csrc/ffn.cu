@@ -71,6 +71,33 @@ __global__ void ffn_link_kernel(const float* __restrict__ inv_s, const int32_t* 
   inv_s_perm[c] = inv_s[j];
 }
 
+// dst row r = src row rows[r] for r < n (rows past n, the padding, copied in
+// place); rows of row_vecs 16-byte vectors
+__global__ void permute_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                    const int32_t* __restrict__ rows, int64_t n, int64_t nrows,
+                                    int64_t row_vecs) {
+  const int64_t total = nrows * row_vecs;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / row_vecs, c = i - r * row_vecs;
+    const int64_t from = r < n ? rows[r] : r;
+    dst[r * row_vecs + c] = src[from * row_vecs + c];
+  }
+}
+
+// the same for the E8M0 scale bytes, which sit in the MMA's atom layout
+__global__ void permute_sf_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                  const int32_t* __restrict__ rows, int64_t n, int64_t nrows,
+                                  int64_t nblk) {
+  const int64_t total = nrows * nblk;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nblk, b = i - r * nblk;
+    const int64_t from = r < n ? rows[r] : r;
+    dst[sf_offset(r, b, nblk)] = src[sf_offset(from, b, nblk)];
+  }
+}
+
 }  // namespace w4a4
 
 using namespace w4a4;
@@ -153,4 +180,33 @@ extern "C" w4a4_status w4a4_gemm_dual_act(const uint8_t* aq, const uint8_t* sfa,
   act.k_pad = gn.k_pad;
   return from_cuda(launch_gemm(aq, sfa, xo, T, g, pw->wq, pw->sfb, pw->w_hp, nullptr, g.d_out, s,
                                &act));
+}
+
+extern "C" w4a4_status w4a4_permute_packed_rows(const w4a4_packed_weight* src, const int32_t* rows,
+                                                const w4a4_packed_weight* dst, void* stream) {
+  Geometry g, gd;
+  w4a4_status st = check_pw(src, &g);
+  if (st != W4A4_OK) return st;
+  st = check_pw(dst, &gd);
+  if (st != W4A4_OK) return st;
+  if (rows == nullptr || src->d_in != dst->d_in || src->d_out != dst->d_out || src->k != dst->k ||
+      src->layout != dst->layout)
+    return W4A4_ERR_INVALID_ARG;
+  if ((g.kj > 0 && (src->wq == dst->wq || src->sfb == dst->sfb)) ||
+      (g.k > 0 && src->w_hp == dst->w_hp))
+    return W4A4_ERR_INVALID_ARG;                       // not in place
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = device_num_sms() > 0 ? device_num_sms() : 148;
+  const int grid = 4 * sms;
+  if (g.kj > 0) {
+    permute_rows_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(src->wq),
+                                             reinterpret_cast<uint4*>(dst->wq), rows, g.d_out,
+                                             g.d_out, g.kj_pad / 2 / 16);
+    permute_sf_kernel<<<grid, 256, 0, s>>>(src->sfb, dst->sfb, rows, g.d_out, g.sfb_rows, g.nblk);
+  }
+  if (g.k > 0)
+    permute_rows_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(src->w_hp),
+                                             reinterpret_cast<uint4*>(dst->w_hp), rows, g.d_out,
+                                             g.d_out, g.k_pad * 2 / 16);
+  return cudaGetLastError() == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }

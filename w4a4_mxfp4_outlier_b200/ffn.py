@@ -2,8 +2,8 @@
 
 The review quantises both FFN projections of the Wan2.2 DiT with the same
 recipe (sec. 3.1, 3.5).  calibrate_ffn builds both packed layers; with the
-up layer's weight rows stored in the down layer's compacted input order
-(w4a4_ffn_link / w4a4_pack_weight_rows), forward() runs
+up layer's packed rows reordered into the down layer's compacted input order
+(w4a4_ffn_link / w4a4_permute_packed_rows), forward() runs
 
     prep_act(X) -> gemm_dual_act (up; its epilogue applies GELU and the down
     layer's activation prep) -> gemm_dual (down)
@@ -20,7 +20,7 @@ from dataclasses import dataclass
 import torch
 
 from . import (PackedWeight, SF_32x1_KMAJOR, _check, _ffn_link, _gelu_bf16, _gemm_dual_act, _nz,
-               _pack_weight_rows, _ptr, _stream, ActBuffers, alloc_act, alloc_packed, calib_finalize,
+               _permute_packed_rows, _ptr, _stream, ActBuffers, alloc_act, alloc_packed, calib_finalize,
                calib_observe, calibrate, gemm_dual, linear, pack_weight, prep_act, workspace_size)
 
 
@@ -69,8 +69,11 @@ def calibrate_ffn(X_batches, W_up: torch.Tensor, W_down: torch.Tensor, alpha_up:
     up.s, up.inv_s, up.score, up.O, up.jmap = (up_plain.s, up_plain.inv_s, up_plain.score,
                                                up_plain.O, up_plain.jmap)
     up.act_scale, up.w_scale = up_plain.act_scale, up_plain.w_scale
-    _check(_pack_weight_rows(_ptr(W_up), W_up.stride(0), _ptr(up.s), _ptr(perm), ctypes.byref(up.c),
-                             _stream(stream)), "pack_weight_rows")
+    # reorder the natural pack (not a pack of the reordered W): every output
+    # channel keeps its quantisation, 32x32 tiles included, so the fused and
+    # unfused FFN compute the same function
+    _check(_permute_packed_rows(ctypes.byref(up_plain.c), _ptr(perm), ctypes.byref(up.c),
+                                _stream(stream)), "permute_packed_rows")
     return PackedFFN(up, down, perm, inv_s_perm, up_plain)
 
 

@@ -114,3 +114,35 @@ def test_random_ffn_parity(case):
         np.testing.assert_array_equal(gu.sf_canonical(act_down.sfa, T, d.nblk, nb)[:, :nb], ref["sfa"])
     if k_down:
         np.testing.assert_array_equal(gu.bf16_bits(act_down.xo)[:, :k_down], ref["xo"])
+
+
+@pytest.mark.parametrize("L", _cases()[::4], ids=lambda L: L.name)
+def test_random_shape_variants(L):
+    """The same layer through the other entry points gives the same bits as
+    linear: a checkpoint round trip, the no-allocation entry point (where the
+    problem fits its scratch array) and strided X and Y rows."""
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
+    ws = torch.empty(w4.workspace_size(L.T, L.d_in, L.d_out, L.k), dtype=torch.uint8, device="cuda")
+    Y = torch.empty((L.T, L.d_out), dtype=torch.bfloat16, device="cuda")
+    w4.linear(X, pw, ws, Y)
+    # checkpoint round trip
+    pl = w4.packed_from_bytes(w4.packed_to_bytes(pw))
+    Y2 = torch.empty_like(Y)
+    w4.linear(X, pl, ws, Y2)
+    # strided rows
+    Xs = torch.zeros((L.T, L.d_in + 24), dtype=torch.bfloat16, device="cuda")
+    Xs[:, :L.d_in] = X
+    Ys = torch.zeros((L.T, L.d_out + 48), dtype=torch.bfloat16, device="cuda")
+    w4.linear(Xs[:, :L.d_in], pw, ws, Ys[:, :L.d_out])
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    assert torch.equal(Y.view(torch.int16), Ys[:, :L.d_out].contiguous().view(torch.int16))
+    assert not Ys[:, L.d_out:].any()
+    if ws.numel() <= w4.NOALLOC_SCRATCH_BYTES:
+        Y3 = torch.empty_like(Y)
+        w4.linear_noalloc(X, pw, Y3)
+        torch.cuda.synchronize()
+        assert torch.equal(Y.view(torch.int16), Y3.view(torch.int16))
+    st, bits = w4.last_error()
+    assert st == w4.OK, hex(bits)

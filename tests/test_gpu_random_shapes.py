@@ -146,3 +146,41 @@ def test_random_shape_variants(L):
         assert torch.equal(Y.view(torch.int16), Y3.view(torch.int16))
     st, bits = w4.last_error()
     assert st == w4.OK, hex(bits)
+
+
+def _topk_cases(n=30, seed=5):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        d_in = int(rng.integers(1, 2049)) * 8
+        k = int(rng.choice([0, 1, 2, 31, 64, 257, d_in // 2, d_in - 1, d_in]))
+        k = max(0, min(k, d_in))
+        nvals = int(rng.choice([1, 2, 3, 17, 1000]))
+        out.append((f"topk{i}_d{d_in}_k{k}_v{nvals}", d_in, k, nvals, 300 + i))
+    return out
+
+
+@pytest.mark.parametrize("case", _topk_cases(), ids=lambda c: c[0])
+def test_random_topk_with_ties(case):
+    """The device top-k (radix select, ties to the lower column) against the
+    oracle's stable sort, on scores with many exact ties: with alpha = 0.5 and
+    weight magnitudes equal to the activation magnitudes, s = 1 and the score
+    is the activation magnitude itself."""
+    _, d_in, k, nvals, seed = case
+    rng = np.random.default_rng(seed)
+    vals = np.concatenate([[0.0], rng.uniform(1e-3, 50.0, nvals - 1)]).astype(np.float32)
+    act = torch.from_numpy(vals[rng.integers(0, nvals, d_in)]).cuda()
+    wsc = act.clone()
+    f = lambda: torch.empty(d_in, device="cuda")
+    s, inv_s, score = f(), f(), f()
+    O = torch.empty(max(k, 1), dtype=torch.int32, device="cuda")
+    J = torch.empty(max(d_in - k, 1), dtype=torch.int32, device="cuda")
+    w4.calib_finalize(act, wsc, 0.5, k, s, inv_s, score, O if k else None, J if k < d_in else None)
+    torch.cuda.synchronize()
+    sc = score.cpu().numpy()
+    assert np.array_equal(sc, act.cpu().numpy())
+    Oref, Jref = orc.select_outliers(sc, k)
+    if k:
+        np.testing.assert_array_equal(O.cpu().numpy()[:k], Oref)
+    if k < d_in:
+        np.testing.assert_array_equal(J.cpu().numpy()[:d_in - k], Jref)

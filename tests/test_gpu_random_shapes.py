@@ -184,3 +184,34 @@ def test_random_topk_with_ties(case):
         np.testing.assert_array_equal(O.cpu().numpy()[:k], Oref)
     if k < d_in:
         np.testing.assert_array_equal(J.cpu().numpy()[:d_in - k], Jref)
+
+
+def test_prep_special_values():
+    """Prep of rows that are all zero, subnormal, huge (near the bf16 maximum
+    after smoothing) or mixed in sign and magnitude, with a layer calibrated
+    on ordinary data: codes, scales and outliers bit for bit."""
+    L = synth.Layer("special", 64, 512, 256, 0.5, 12, 0, synth.XSpec("student3", 0.3, 6, 8.0, 30.0),
+                    synth.WSpec(0.02), seed=21)
+    X, W = gu.gen(L)
+    pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
+    rng = np.random.default_rng(9)
+    rows = []
+    rows.append(np.zeros(512))                                         # all zero
+    rows.append(np.full(512, -0.0))                                    # negative zeros
+    rows.append(rng.choice([-1, 1], 512) * 2.0 ** rng.integers(-133, -126, 512))   # bf16 subnormals
+    rows.append(rng.choice([-1, 1], 512) * rng.uniform(1e30, 3e33, 512))           # huge
+    rows.append(np.where(rng.random(512) < 0.5, 0.0, rng.normal(0, 1e-20, 512)))   # tiny, sparse
+    rows.append(rng.normal(0, 1, 512) * 10.0 ** rng.integers(-30, 30, 512))        # wild magnitudes
+    while len(rows) < 64:
+        rows.append(rng.normal(0, 0.3, 512))
+    Xs = torch.from_numpy(np.stack(rows).astype(np.float32)).to(torch.bfloat16).cuda()
+    act = w4.alloc_act(64, pw)
+    w4.prep_act(Xs, pw, act)
+    torch.cuda.synchronize()
+    c = gu.oracle_calib_from_gpu(pw)
+    ref = orc.prep_activation(gu.to_np_f32(Xs), c["inv_s"], c["O"], c["J"])
+    d = pw.dims
+    nb = ref["sfa"].shape[1]
+    np.testing.assert_array_equal(act.aq.cpu().numpy()[:, :nb * 16], ref["aq"])
+    np.testing.assert_array_equal(gu.sf_canonical(act.sfa, 64, d.nblk, nb)[:, :nb], ref["sfa"])
+    np.testing.assert_array_equal(gu.bf16_bits(act.xo)[:, :L.k], ref["xo"])

@@ -30,6 +30,12 @@
 // error word and an abort flag the others poll, and all roles then exit
 // through the same teardown (drain in-flight copies / MMAs, free tensor
 // memory).
+//
+// Two kernels follow: gemm_dual_kernel (one CTA per 128 x 256 tile, for
+// T <= 128) and gemm_dual_pair_kernel (a CTA pair per 256 x 256 tile, see its
+// own comment).  Both take a flag kAct: with it, the epilogue does not store
+// Y but runs the fused FFN step (act_block: GELU, the next layer's smoothing
+// and MXFP4 encoding) and writes the next layer's activation buffers.
 #include <cuda.h>
 
 #include "w4a4_internal.h"

@@ -451,12 +451,7 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
-            "config": {"workload": f"{args.workload}: " + ", ".join(
-                f"{L.name} T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
-                f"{LAYOUT_NAMES[L.layout]}" for L in layers),
-                "tokens_per_gpu": layers[0].T, "parallelism": f"token shards x{world}",
-                "l2": "inputs larger than L2 (no flush)",
-                "step": "calib absmax X,W + finalize + pack + prep + dual GEMM per layer"},
+            "config": layer_workload_config(args.workload, layers, world),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -609,12 +604,34 @@ def cpu_baseline(layers, runs=None, rows=64, outs=256):
                       f"(calibrate, pack, prep, product) in numpy; {secs:.1f} s"}
 
 
+def layer_workload_config(workload, layers, world):
+    """The `config` of a layer workload's JSON line (both arms print the same)."""
+    return {"workload": f"{workload}: " + ", ".join(
+                f"{L.name} T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
+                f"{LAYOUT_NAMES[L.layout]}" for L in layers),
+            "tokens_per_gpu": layers[0].T, "parallelism": f"token shards x{world}",
+            "l2": "inputs larger than L2 (no flush)",
+            "step": "calib absmax X,W + finalize + pack + prep + dual GEMM per layer"}
+
+
+def ffn_workload_config(workload, Lu, Ld, world):
+    """The `config` of an FFN workload's JSON line (both arms print the same)."""
+    return {"workload": f"{workload}: T={Lu.T} {Lu.d_in}->{Lu.d_out} k={Lu.k} alpha={Lu.alpha}, GELU, "
+                        f"{Lu.d_out}->{Lu.d_in} k={Ld.k} alpha={Ld.alpha}, {LAYOUT_NAMES[Lu.layout]}",
+            "tokens_per_gpu": Lu.T, "parallelism": f"token shards x{world}",
+            "l2": "inputs larger than L2 (no flush)",
+            "step": "online FFN forward, fused: prep + up GEMM with GELU/prep epilogue "
+                    "+ down GEMM (packed weights prepared before timing)"}
+
+
 def run_reference(args):
     import synth
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    layers = list(synth.WORKLOADS[args.workload])
+    # the FFN workloads: the same two layers, each sampled on its own input
+    name = {"ffn": "full", "ffn_mid": "mid_up"}.get(args.workload, args.workload)
+    layers = list(synth.WORKLOADS[name]) if name != "mid_up" else [synth.MID_UP, synth.MID_DOWN]
     Xs, Ws = _host_samples(layers, None, 64, 256)
     for _ in range(args.warmup):
         oracle_sample(layers, 64, 256, Xs, Ws)
@@ -627,11 +644,17 @@ def run_reference(args):
     cores = _threads_used()
     sample = ("64 token rows x 256 output channels per layer of the workload, whole path "
               "(calibrate, pack, prep, product) in the numpy oracle")
+    if args.workload in ("ffn", "ffn_mid"):
+        sample += ("; the FFN's up and down layers each on its own synthetic input (the GELU "
+                   "between them is not part of the sample)")
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 8), "unit": "TFLOPS",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(tot_s / args.steps * 1e3, 2), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (numpy oracle)",
-           "data": "synthetic", "config": {"workload": args.workload},
+           "data": "synthetic",
+           "config": (ffn_workload_config(args.workload, layers[0], layers[1], world)
+                      if args.workload in ("ffn", "ffn_mid")
+                      else layer_workload_config(args.workload, layers, world)),
            "cpu_baseline": {"value": round(v, 8), "unit": "TFLOPS", "cores": cores,
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(v, 8), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
@@ -736,13 +759,7 @@ def run_ffn(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
-            "config": {"workload": f"{args.workload}: T={T} {d_model}->{d_ff} k={Lu.k} alpha={Lu.alpha}, GELU, "
-                                   f"{d_ff}->{d_model} k={Ld.k} alpha={Ld.alpha}, "
-                                   f"{LAYOUT_NAMES[Lu.layout]}",
-                       "tokens_per_gpu": T, "parallelism": f"token shards x{world}",
-                       "l2": "inputs larger than L2 (no flush)",
-                       "step": "online FFN forward, fused: prep + up GEMM with GELU/prep epilogue "
-                               "+ down GEMM (packed weights prepared before timing)"},
+            "config": ffn_workload_config(args.workload, Lu, Ld, world),
             "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,

@@ -70,6 +70,9 @@ def test_reference_arm_prints_on_rank0_only(monkeypatch):
         bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
     line = json.loads(buf.getvalue().strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["warmup"] == 3
+    # the same config the GPU arm prints for this workload
+    import synth
+    assert line["config"] == bench.layer_workload_config("tiny", synth.WORKLOADS["tiny"], 1)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
 

@@ -271,9 +271,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "bdc61dd4ac7910c5bbbdb2ee73ec00021bf52707ab3cb1b013b449de54c91425",
+    "sha256": "a9d6a62fcb2cca79e01b7471013c4a342d0a63a537c74e446e75e6fb1e6650b5",
     "workload": "full",
-    "bytes_per_launch": (723234560 + 1563205888 + 1461546240 + 573794048) / 2,
+    "bytes_per_launch": (723791360 + 1562562816 + 1210304768 + 574054656) / 2,
 }
 
 

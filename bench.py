@@ -389,6 +389,8 @@ def run_gpu(args):
     mk = lambda: torch.cuda.Event(enable_timing=True)
     evs = [[{"off": [mk(), mk()], "on": [mk(), mk(), mk()]} for _ in runs] for _ in range(args.steps)]
     t0, t1 = mk(), mk()
+    flush = l2_flush_buffer(min(layer_input_bytes(L) for L in layers), device)
+    s_evs = [(mk(), mk()) for _ in range(args.steps)]
     clocks = clock_sampler(local)
     torch.cuda.synchronize()
     dist_barrier(active, device)
@@ -398,7 +400,11 @@ def run_gpu(args):
     t0.record()
     launches = 0
     for k in range(args.steps):
+        if flush is not None:
+            flush.zero_()                       # between steps, outside the step's events
+        s_evs[k][0].record()
         launches += step(evs[k])
+        s_evs[k][1].record()
     t1.record()
     torch.cuda.synchronize()
     clocks.mark_end()
@@ -408,7 +414,7 @@ def run_gpu(args):
     if st != w4.OK:
         raise RuntimeError(f"device error word {bits:#x} in the timed region")
 
-    step_ms = t0.elapsed_time(t1) / args.steps
+    step_ms = sum(a.elapsed_time(b) for a, b in s_evs) / args.steps
     step_ms_max = dist_max(step_ms, active, device)
     flops = sum(L.flops for L in layers)
     value = aggregate(flops, world, step_ms_max * 1e-3) / 1e12
@@ -451,7 +457,7 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
-            "config": layer_workload_config(args.workload, layers, world),
+            "config": layer_workload_config(args.workload, layers, world, flush is not None),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -604,22 +610,53 @@ def cpu_baseline(layers, runs=None, rows=64, outs=256):
                       f"(calibrate, pack, prep, product) in numpy; {secs:.1f} s"}
 
 
-def layer_workload_config(workload, layers, world):
+L2_BYTES = 126e6     # B200 L2
+
+
+def layer_input_bytes(L) -> float:
+    """A layer step's inputs: X and W, bf16."""
+    return 2.0 * (L.T * L.d_in + L.d_out * L.d_in)
+
+
+def l2_flush_buffer(input_bytes: float, device):
+    """A 256 MB buffer to overwrite L2 between timed steps when a step's inputs
+    are under twice the L2 size, else None (the inputs flush it themselves)."""
+    if input_bytes >= 2 * L2_BYTES:
+        return None
+    import torch
+    return torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+
+def l2_note(flushed: bool) -> str:
+    return ("L2 flushed between steps: 256 MB written outside the steps' events" if flushed
+            else "inputs larger than L2 (no flush)")
+
+
+def layer_workload_config(workload, layers, world, flushed=None):
     """The `config` of a layer workload's JSON line (both arms print the same)."""
+    if flushed is None:
+        flushed = min(layer_input_bytes(L) for L in layers) < 2 * L2_BYTES
     return {"workload": f"{workload}: " + ", ".join(
                 f"{L.name} T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
                 f"{LAYOUT_NAMES[L.layout]}" for L in layers),
             "tokens_per_gpu": layers[0].T, "parallelism": f"token shards x{world}",
-            "l2": "inputs larger than L2 (no flush)",
+            "l2": l2_note(flushed),
             "step": "calib absmax X,W + finalize + pack + prep + dual GEMM per layer"}
 
 
-def ffn_workload_config(workload, Lu, Ld, world):
+def ffn_input_bytes(Lu) -> float:
+    """An FFN step's input: X, bf16 (the weights are packed before timing)."""
+    return 2.0 * Lu.T * Lu.d_in
+
+
+def ffn_workload_config(workload, Lu, Ld, world, flushed=None):
     """The `config` of an FFN workload's JSON line (both arms print the same)."""
+    if flushed is None:
+        flushed = ffn_input_bytes(Lu) < 2 * L2_BYTES
     return {"workload": f"{workload}: T={Lu.T} {Lu.d_in}->{Lu.d_out} k={Lu.k} alpha={Lu.alpha}, GELU, "
                         f"{Lu.d_out}->{Lu.d_in} k={Ld.k} alpha={Ld.alpha}, {LAYOUT_NAMES[Lu.layout]}",
             "tokens_per_gpu": Lu.T, "parallelism": f"token shards x{world}",
-            "l2": "inputs larger than L2 (no flush)",
+            "l2": l2_note(flushed),
             "step": "online FFN forward, fused: prep + up GEMM with GELU/prep epilogue "
                     "+ down GEMM (packed weights prepared before timing)"}
 
@@ -720,7 +757,9 @@ def run_ffn(args):
         raise RuntimeError("fused and unfused FFN outputs differ")
 
     evs = [[mk() for _ in range(4)] for _ in range(args.steps)]
-    t0, t1, u0, u1 = mk(), mk(), mk(), mk()
+    t0, t1 = mk(), mk()
+    u_evs = [(mk(), mk()) for _ in range(args.steps)]
+    flush = l2_flush_buffer(ffn_input_bytes(Lu), device)
     clocks = clock_sampler(local)
     torch.cuda.synchronize()
     dist_barrier(active, device)
@@ -730,20 +769,24 @@ def run_ffn(args):
     t0.record()
     launches = 0
     for k in range(args.steps):
+        if flush is not None:
+            flush.zero_()                       # between steps, outside the step's events
         launches += fused(evs[k])
     t1.record()
     torch.cuda.synchronize()
     clocks.mark_end()
     clock_info = clocks.stop()
-    u0.record()
-    for _ in range(args.steps):
+    for k in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        u_evs[k][0].record()
         unfused()
-    u1.record()
+        u_evs[k][1].record()
     torch.cuda.synchronize()
     dist_barrier(active, device)
-    step_ms = t0.elapsed_time(t1) / args.steps
+    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
     step_ms_max = dist_max(step_ms, active, device)
-    unfused_ms = u0.elapsed_time(u1) / args.steps
+    unfused_ms = sum(a.elapsed_time(b) for a, b in u_evs) / args.steps
     flops = 2.0 * (2.0 * T * d_model * d_ff)
     value = aggregate(flops, world, step_ms_max * 1e-3) / 1e12
     avg = lambda i, j: sum(e[i].elapsed_time(e[j]) for e in evs) / args.steps
@@ -759,7 +802,7 @@ def run_ffn(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1/e8m0 x e2m1/e8m0 + bf16 x bf16, f32 accumulate",
             "data": "synthetic (seeded heavy-tailed X, clipped-normal W; see synth/)",
-            "config": ffn_workload_config(args.workload, Lu, Ld, world),
+            "config": ffn_workload_config(args.workload, Lu, Ld, world, flush is not None),
             "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,

@@ -80,6 +80,18 @@ def test_reference_arm_prints_on_rank0_only(monkeypatch):
 
 
 
+def test_l2_flush_only_where_inputs_fit_in_twice_l2():
+    import synth
+    flushed = lambda w: bench.layer_workload_config(w, synth.WORKLOADS[w], 1)["l2"].startswith("L2 flushed")
+    # X_up alone is 590 MB and X_down 1.6 GB: no flush needed on the full layers
+    assert not flushed("full") and not flushed("full_up") and not flushed("full_down")
+    assert flushed("tiny")
+    # X 168 MB + W 142 MB reach twice the 126 MB L2; the FFN step reads X alone
+    assert not bench.layer_input_bytes(synth.MID_UP) < 2 * bench.L2_BYTES
+    assert bench.ffn_workload_config("ffn_mid", synth.MID_UP, synth.MID_DOWN, 1)["l2"].startswith("L2 flushed")
+    assert bench.l2_flush_buffer(bench.layer_input_bytes(synth.WORKLOADS["full"][0]), None) is None
+
+
 def test_peak_choice_by_timed_region_length():
     assert bench.peak_keys(0.04) == ("bf16_tflops", "bf16_tflops_sustained")
     assert bench.peak_keys(1.5) == ("bf16_tflops_sustained", "bf16_tflops")

@@ -271,9 +271,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "a9d6a62fcb2cca79e01b7471013c4a342d0a63a537c74e446e75e6fb1e6650b5",
+    "sha256": "d22c666630c87ef5a0a7612f6398c7c9b8cae53e6ad83c7e0ad292eb189538f5",
     "workload": "full",
-    "bytes_per_launch": (723791360 + 1562562816 + 1210304768 + 574054656) / 2,
+    "bytes_per_launch": (737091840 + 1560132352 + 1584012800 + 572660736) / 2,
 }
 
 
@@ -357,6 +357,28 @@ class LayerRun:
         if ev is not None:
             ev[2].record()
         return 2
+
+
+def cublas_bf16_context(runs, reps=5):
+    """cuBLAS bf16 GEMM of the same shapes (Y = X W^T through torch.mm), timed
+    after the timed region as context: the unquantised product this path
+    replaces.  Returns the mean milliseconds per layer."""
+    import torch
+    out = []
+    for r in runs:
+        Yc = torch.empty_like(r.Y)
+        for _ in range(2):
+            torch.mm(r.X, r.W.t(), out=Yc)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            torch.mm(r.X, r.W.t(), out=Yc)
+        b.record()
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b) / reps)
+        del Yc
+    return out
 
 
 def run_gpu(args):
@@ -445,6 +467,7 @@ def run_gpu(args):
             "frac_of_other_peak": round(gemm_tflops / other, 4),
             "frac_of_nominal_fp4_9pf": round(gemm_tflops / FP4_NOMINAL_TFLOPS, 4)}
 
+    cublas_ms = cublas_bf16_context(runs)
     e2e = run_e2e(args, runs, w4, device, active) if not args.no_e2e else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -474,6 +497,12 @@ def run_gpu(args):
                 "calib_absmax_gbs": round(calib_bytes / (sum(calib_ms) * 1e-3) / 1e9, 1),
                 "online_tflops": round(online_tflops, 1),
             },
+            "context_cublas_bf16": {
+                "gemm_ms": [round(x, 4) for x in cublas_ms],
+                "tflops": round(flops / (sum(cublas_ms) * 1e-3) / 1e12, 1),
+                "dual_gemm_speedup": round(sum(cublas_ms) / sum(gemm_ms), 3),
+                "note": "torch.mm bf16 of the same X and W, timed after the timed region "
+                        "(5 reps, L2 not flushed); not part of the step"},
         }
         print(json.dumps(out), flush=True)
     if active:

@@ -39,6 +39,16 @@ MID128 = MID.with_(name="mid_k64_128x1", layout=2, k=64)
 
 SMALL = [TINY, RAGGED, RAGGED32, RAGGED128, K0, KFULL, T1, SINGLE]
 
+# the 384-column pair tile (d_out a multiple of 384, T > 128): ragged M tile,
+# ragged last bf16 K tile (k = 37), one to three N tiles, all three weight
+# scale layouts, no MXFP4 columns at all (k = d_in) and no outliers (k = 0)
+TILE384 = [
+    synth.Layer("tile384_T300_k37", 300, 1024, 768, 0.6, 37, 0, synth.X_UP, synth.W_UP),
+    synth.Layer("tile384_T129_32x32_k0", 129, 512, 1152, 0.5, 0, 1, synth.X_UP, synth.W_UP),
+    synth.Layer("tile384_T520_128x1_k64", 520, 2048, 384, 0.7, 64, 2, synth.X_UP, synth.W_UP),
+    synth.Layer("tile384_kfull", 300, 64, 384, 0.5, 64, 0, synth.X_TINY, synth.WSpec(0.02)),
+]
+
 # the prep kernel's launch shapes: block-per-lane form with 2 thread groups
 # (192 blocks; with the 6-slot ring at d_in 6144 and the 18-slot ring for
 # short rows at 5440; 6 and 3 groups on short rows are the small shapes and
@@ -239,7 +249,7 @@ def _linear(X, pw, T, d_out):
     return Y
 
 
-@pytest.mark.parametrize("L", SMALL + [MID, MID128], ids=lambda L: L.name)
+@pytest.mark.parametrize("L", SMALL + [MID, MID128] + TILE384, ids=lambda L: L.name)
 def test_linear_parity_full_output(L):
     X, W, pw = _calibrate(L)
     Y = _linear(X, pw, L.T, L.d_out)

@@ -36,7 +36,24 @@ def _cases(n=80, seed=2024):
     return out
 
 
-@pytest.mark.parametrize("L", _cases(), ids=lambda L: L.name)
+def _cases384(n=16, seed=2025):
+    """Shapes that run on the 384-column pair tile: d_out a multiple of 384, T > 128."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        T = int(rng.choice([129, 200, 256, 257, 511, 700]))
+        d_in = int(rng.integers(1, 400)) * 8
+        d_out = int(rng.integers(1, 5)) * 384
+        k = min(int(rng.choice([0, 1, 17, 64, 100, d_in])), d_in)
+        layout = int(rng.integers(0, 3))
+        alpha = float(rng.choice([0.4, 0.6, 0.7]))
+        xs = synth.XSpec("student3", 0.3, int(min(d_in, rng.integers(0, 16))), 8.0, 30.0)
+        out.append(synth.Layer(f"rand384_{i}_T{T}_{d_in}x{d_out}_k{k}_l{layout}", T, d_in, d_out,
+                               alpha, k, layout, xs, synth.WSpec(0.02), seed=300 + i))
+    return out
+
+
+@pytest.mark.parametrize("L", _cases() + _cases384(), ids=lambda L: L.name)
 def test_random_shape_parity(L):
     X, W = gu.gen(L)
     pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)

@@ -32,11 +32,14 @@
 // memory).
 //
 // Two kernels follow: gemm_dual_kernel (one CTA per 128 x 256 tile, for
-// T <= 128) and gemm_dual_pair_kernel (a CTA pair per 256 x 256 tile, see its
-// own comment).  Both take a flag kAct: with it, the epilogue does not store
+// T <= 128) and gemm_dual_pair_kernel (a CTA pair per 256 x 256 or 256 x 384
+// tile, see its own comment; its tensor-memory columns differ).  Both take a flag kAct: with it, the epilogue does not store
 // Y but runs the fused FFN step (act_block: GELU, the next layer's smoothing
 // and MXFP4 encoding) and writes the next layer's activation buffers.
 #include <cuda.h>
+
+#include <cstdlib>
+#include <cstring>
 
 #include "w4a4_internal.h"
 
@@ -474,12 +477,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
 // ===========================================================================
 // CTA-pair kernel (tcgen05 cta_group::2): a cluster of two CTAs computes a
-// 256 x 256 output tile.  CTA r of the pair stages its own 128 token rows of
-// A and its own 128 output rows of B (so B's shared-memory traffic per SM
-// halves against the single-CTA kernel), plus its A scales and all 256 rows of
-// B scales; the leader CTA (rank 0) issues the M=256 MMAs for both.  Each
-// CTA's tensor memory holds the accumulator of its 128 rows and, in the same
-// layout as the single-CTA kernel, its scale factors.
+// 256 x kN output tile, kN = 256 or 384.  CTA r of the pair stages its own
+// 128 token rows of A and its own half of the tile's B rows (so B's
+// shared-memory traffic per SM halves against the single-CTA kernel), plus
+// its A scales and the scales of all kN rows of B; the leader CTA (rank 0)
+// issues the M=256 MMAs for both.  Each CTA's tensor memory holds the
+// accumulator of its 128 rows (kN columns) and its scale factors.
+//
+// kN = 384 (plain epilogue only): each K step is one N=256 MMA into columns
+// 0..255 and one N=128 MMA into columns 256..383 with the same A.  A is then
+// fed once per 384 output columns instead of per 256 (a third fewer operand
+// bytes per FLOP from A) and there are a third fewer tile hand-offs between
+// the MMA issuer and the epilogue.  Per CTA and K tile, B is 128 rows for the
+// first MMA (rows 128r .. 128r+127 of the tile) and 64 for the second (rows
+// 256+64r .. 256+64r+63), stacked in shared memory; the tile's 384 scale rows
+// are three 128-row atoms.
 //
 // Synchronisation: the TMA copies of both CTAs complete on the leader's
 // "full" barrier (the leader posts the expected byte count of both); the
@@ -487,24 +499,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // barriers of both CTAs; the epilogue warps of both CTAs arrive on the
 // leader's "acc_empty".  No load uses cluster multicast.
 // ===========================================================================
-constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = 128 * KT_BYTES;     // own 128 token rows
-constexpr int P_B_BYTES = 128 * KT_BYTES;     // own 128 output rows
 constexpr int P_SFA_BYTES = 1024;             // own 128 rows x 8 blocks
-constexpr int P_SFB_BYTES = 2048;             // all 256 output rows x 8 blocks
-constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;
 constexpr int P_EPI_ARRIVALS = 2 * NUM_EPI_WARPS;
 
 constexpr int P_EPI_BYTES = 16 * 64;          // staging block: 16 rows x 32 bf16 (64-byte swizzle)
 
-// The plain kernel: 6 stages, a 1 KB Y staging block per epilogue warp.  The
-// fused FFN kernel: 5 stages, a 2 KB block per warp (its 32 rows x 64 code
-// bytes of one tile half) and the GELU table.
-template <bool kAct>
+// Per tile width kN: B rows per CTA (kN / 2), B scale bytes (all kN rows x 8
+// blocks), stage bytes, pipeline depth (about 1.6 us of MMA work either way)
+// and tensor-memory columns of the scale buffers (after the accumulator).
+template <int kN>
+struct PairTile {
+  static_assert(kN == 256 || kN == 384, "pair tile width");
+  static constexpr int kBBytes = (kN / 2) * KT_BYTES;
+  static constexpr int kSfbBytes = (kN / 128) * 1024;
+  static constexpr int kStageBytes = P_A_BYTES + kBBytes + P_SFA_BYTES + kSfbBytes;
+  static constexpr int kStages = kN == 256 ? 6 : 4;
+  static constexpr int kSfaCol = kN;                 // 2 atoms x 4 columns
+  static constexpr int kSfbCol = kN + 8;             // 2 atoms x 8 columns (first 256 rows)
+  static constexpr int kSfb2Col = kN + 24;           // 2 atoms x 4 columns (rows 256..383)
+  static constexpr int kSfBuf = kN == 256 ? 32 : 48; // scale buffers alternate by K tile
+  static_assert(kSfb2Col + 8 + kSfBuf <= TMEM_COLS, "tensor memory columns");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+};
+
+// The plain kernel: PairTile stages, a 1 KB Y staging block per epilogue
+// warp.  The fused FFN kernel (kN = 256): 5 stages, a 2 KB block per warp
+// (its 32 rows x 64 code bytes of one tile half) and the GELU table.
+template <bool kAct, int kN>
 struct PairSmem {
-  static constexpr int kStages = kAct ? 5 : P_STAGES;
+  static_assert(!kAct || kN == 256, "the fused epilogue runs on 256-wide tiles");
+  static constexpr int kStages = kAct ? 5 : PairTile<kN>::kStages;
   static constexpr int kEpiBytes = kAct ? 32 * 64 : P_EPI_BYTES;
-  uint8_t stage[kStages][P_STAGE_BYTES];
+  uint8_t stage[kStages][PairTile<kN>::kStageBytes];
   alignas(1024) uint8_t epi[NUM_EPI_WARPS][kEpiBytes];
   alignas(16) uint16_t gelu_tab[kAct ? kGeluTabEntries : 8];
   uint64_t full[kStages];      // leader's counts the bytes of both CTAs
@@ -516,15 +543,18 @@ struct PairSmem {
   uint32_t abort_flag;
 };
 
-template <bool kAct>
+template <bool kAct, int kN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_dual_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_ao, const __grid_constant__ CUtensorMap tm_bo,
                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                           const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ GemmArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  using Smem = PairSmem<kAct>;
+  using Smem = PairSmem<kAct, kN>;
+  using Tile = PairTile<kN>;
   constexpr int NST = Smem::kStages;
+  constexpr int P_B_BYTES = Tile::kBBytes;
+  constexpr int P_STAGE_BYTES = Tile::kStageBytes;
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   volatile uint32_t* abort_flag = &sm.abort_flag;
@@ -534,7 +564,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t rank = cluster_ctarank();          // 0 = leader
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int ntiles = args.tiles_m * args.tiles_n;   // 256 x 256 tiles
+  const int ntiles = args.tiles_m * args.tiles_n;   // 256 x kN tiles
   const int nkt = args.kt_o + args.kt_j;
 
   if (threadIdx.x == 0) {
@@ -579,7 +609,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int tm, tn;
       tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
       const int m_rows = tm * 256 + 128 * static_cast<int>(rank);
-      const int n_rows = tn * 256 + 128 * static_cast<int>(rank);
+      const int n_rows = tn * kN + 128 * static_cast<int>(rank);
+      const int n_rows2 = tn * kN + 256 + 64 * static_cast<int>(rank);   // kN = 384 only
       for (int kt = 0; kt < nkt; ++kt, ++it) {
         if (it >= NST &&
             !warp_wait_bounded(&sm.empty[s], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
@@ -593,17 +624,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // the leader's barrier expects the bytes of both CTAs
             if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_BYTES + P_B_BYTES));
             tma_load_2d_pair(st, &tm_ao, full_leader, kt * 64, m_rows);
-            tma_load_2d_pair(st + P_A_BYTES, &tm_bo, full_leader, kt * 64, n_rows);
+            if constexpr (kN == 256) {
+              tma_load_2d_pair(st + P_A_BYTES, &tm_bo, full_leader, kt * 64, n_rows);
+            } else {             // B in 64-row boxes: 128 rows, then the 64 of the second MMA
+              tma_load_2d_pair(st + P_A_BYTES, &tm_bo, full_leader, kt * 64, n_rows);
+              tma_load_2d_pair(st + P_A_BYTES + 64 * KT_BYTES, &tm_bo, full_leader, kt * 64,
+                               n_rows + 64);
+              tma_load_2d_pair(st + P_A_BYTES + 128 * KT_BYTES, &tm_bo, full_leader, kt * 64,
+                               n_rows2);
+            }
           } else {
             const int kj = kt - args.kt_o;
             if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * P_STAGE_BYTES);
             tma_load_2d_pair(st, &tm_a, full_leader, kj * KT_BYTES, m_rows);
-            tma_load_2d_pair(st + P_A_BYTES, &tm_b, full_leader, kj * KT_BYTES, n_rows);
+            if constexpr (kN == 256) {
+              tma_load_2d_pair(st + P_A_BYTES, &tm_b, full_leader, kj * KT_BYTES, n_rows);
+            } else {
+              tma_load_2d_pair(st + P_A_BYTES, &tm_b, full_leader, kj * KT_BYTES, n_rows);
+              tma_load_2d_pair(st + P_A_BYTES + 64 * KT_BYTES, &tm_b, full_leader, kj * KT_BYTES,
+                               n_rows + 64);
+              tma_load_2d_pair(st + P_A_BYTES + 128 * KT_BYTES, &tm_b, full_leader, kj * KT_BYTES,
+                               n_rows2);
+            }
             // scale atoms: 256-byte rows of the scale buffers, 4 rows (1 KB) per copy
             const int ya = ((2 * tm + static_cast<int>(rank)) * atoms_k + 2 * kj) * 2;
             tma_load_2d_pair(st + P_A_BYTES + P_B_BYTES, &tm_sfa, full_leader, 0, ya);
-            for (int rb = 0; rb < 2; ++rb) {
-              const int yb = ((2 * tn + rb) * atoms_k + 2 * kj) * 2;
+            for (int rb = 0; rb < kN / 128; ++rb) {
+              const int yb = (((kN / 128) * tn + rb) * atoms_k + 2 * kj) * 2;
               tma_load_2d_pair(st + P_A_BYTES + P_B_BYTES + P_SFA_BYTES + rb * 1024, &tm_sfb,
                                full_leader, 0, yb);
             }
@@ -643,11 +690,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint64_t db0 = sdesc_kmajor_sw128(st0 + P_A_BYTES);
       const uint64_t dsa0 = sdesc_sf_rows16(st0 + P_A_BYTES + P_B_BYTES);
       const uint64_t dsb0 = sdesc_sf_rows16(st0 + P_A_BYTES + P_B_BYTES + P_SFA_BYTES);
+      const uint64_t db1 = sdesc_kmajor_sw128(st0 + P_A_BYTES + 128 * KT_BYTES);   // kN = 384
       constexpr uint32_t ID_O = idesc_bf16(256, 256);
       constexpr uint32_t ID_J0 = idesc_mxf4(256, 256, 0, 0);
       constexpr uint32_t ID_J2 = idesc_mxf4(256, 256, 2, 2);
-      const uint32_t tsfa = tmem + TMEM_SFA_COL;
-      const uint32_t tsfb = tmem + TMEM_SFB_COL;
+      constexpr uint32_t ID_O2 = idesc_bf16(256, 128);
+      constexpr uint32_t ID_K0 = idesc_mxf4(256, 128, 0, 0);
+      constexpr uint32_t ID_K2 = idesc_mxf4(256, 128, 2, 2);
+      const uint32_t tsfa = tmem + Tile::kSfaCol;
+      const uint32_t tsfb = tmem + Tile::kSfbCol;
+      const uint32_t tsfb2 = tmem + Tile::kSfb2Col;
+      const uint32_t tacc2 = tmem + 256;
       const int kt_o = args.kt_o, kt_j = args.kt_j;
       const int nk_last_o = (args.k_pad - (kt_o - 1) * 64) / 16;   // K=16 steps in the last bf16 tile
       uint32_t s = 0, ph = 0, buf = 0, tcount = 0;
@@ -668,8 +721,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           if (elect_one()) {
             const int nk = kt + 1 < kt_o ? 4 : nk_last_o;
-            for (int kk = 0; kk < nk; ++kk)
+            for (int kk = 0; kk < nk; ++kk) {
               mma_bf16_pair(tmem, da0 + soff + 2 * kk, db0 + soff + 2 * kk, ID_O, acc | kk);
+              if constexpr (kN == 384)
+                mma_bf16_pair(tacc2, da0 + soff + 2 * kk, db1 + soff + 2 * kk, ID_O2, acc | kk);
+            }
             tc_commit_pair_multicast(&sm.empty[s], 0x3);
           }
           __syncwarp();
@@ -697,17 +753,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tc_cp_pair_32x128b_warpx4(sb + 8, dsb0 + soff + 32);
             tc_cp_pair_32x128b_warpx4(sb + 4, dsb0 + soff + 64);
             tc_cp_pair_32x128b_warpx4(sb + 12, dsb0 + soff + 96);
-            mma_mxf4_pair(tmem, da0 + soff + 0, db0 + soff + 0, ID_J0, sa, sb, acc);
-            mma_mxf4_pair(tmem, da0 + soff + 2, db0 + soff + 2, ID_J2, sa | (2u << 30),
-                          sb | (2u << 30), 1u);
-            mma_mxf4_pair(tmem, da0 + soff + 4, db0 + soff + 4, ID_J0, sa + 4, sb + 8, 1u);
-            mma_mxf4_pair(tmem, da0 + soff + 6, db0 + soff + 6, ID_J2, (sa + 4) | (2u << 30),
-                          (sb + 8) | (2u << 30), 1u);
+            if constexpr (kN == 384) {
+              // the third 128-row atom of B scales: K atoms 0 and 1 at +0 / +4
+              const uint32_t sc = tsfb2 + buf;
+              tc_cp_pair_32x128b_warpx4(sc + 0, dsb0 + soff + 128);
+              tc_cp_pair_32x128b_warpx4(sc + 4, dsb0 + soff + 160);
+              mma_mxf4_pair(tmem, da0 + soff + 0, db0 + soff + 0, ID_J0, sa, sb, acc);
+              mma_mxf4_pair(tacc2, da0 + soff + 0, db1 + soff + 0, ID_K0, sa, sc, acc);
+              mma_mxf4_pair(tmem, da0 + soff + 2, db0 + soff + 2, ID_J2, sa | (2u << 30),
+                            sb | (2u << 30), 1u);
+              mma_mxf4_pair(tacc2, da0 + soff + 2, db1 + soff + 2, ID_K2, sa | (2u << 30),
+                            sc | (2u << 30), 1u);
+              mma_mxf4_pair(tmem, da0 + soff + 4, db0 + soff + 4, ID_J0, sa + 4, sb + 8, 1u);
+              mma_mxf4_pair(tacc2, da0 + soff + 4, db1 + soff + 4, ID_K0, sa + 4, sc + 4, 1u);
+              mma_mxf4_pair(tmem, da0 + soff + 6, db0 + soff + 6, ID_J2, (sa + 4) | (2u << 30),
+                            (sb + 8) | (2u << 30), 1u);
+              mma_mxf4_pair(tacc2, da0 + soff + 6, db1 + soff + 6, ID_K2, (sa + 4) | (2u << 30),
+                            (sc + 4) | (2u << 30), 1u);
+            } else {
+              mma_mxf4_pair(tmem, da0 + soff + 0, db0 + soff + 0, ID_J0, sa, sb, acc);
+              mma_mxf4_pair(tmem, da0 + soff + 2, db0 + soff + 2, ID_J2, sa | (2u << 30),
+                            sb | (2u << 30), 1u);
+              mma_mxf4_pair(tmem, da0 + soff + 4, db0 + soff + 4, ID_J0, sa + 4, sb + 8, 1u);
+              mma_mxf4_pair(tmem, da0 + soff + 6, db0 + soff + 6, ID_J2, (sa + 4) | (2u << 30),
+                            (sb + 8) | (2u << 30), 1u);
+            }
             tc_commit_pair_multicast(&sm.empty[s], 0x3);
           }
           __syncwarp();
           acc = 1;
-          buf ^= TMEM_SF_BUF;
+          buf ^= Tile::kSfBuf;
           if (++s == NST) {
             s = 0;
             ph ^= 1u;
@@ -749,6 +824,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
       if (!ready) break;
       tc_fence_after();
+      if constexpr (kN == 384) {
+        // this warp's 32 rows x 192 columns, converted to bf16 pairs 16
+        // columns at a time so the registers hold 96 words (not 192) plus
+        // one 16-column load; the accumulator is released once all are in
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sp) << 16) + 192 * half;
+        BfPairs16 yb[6];
+#pragma unroll
+        for (int h = 0; h < 12; ++h) {
+          uint32_t r1[16];
+          tmem_ld_32x32b_x16(taddr + 16 * h, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat162 b2 =
+                __floats2bfloat162_rn(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+            yb[h >> 1].w[8 * (h & 1) + j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * sp;
+        const uint32_t stg = smem_u32(sm.epi[ew]);
+#pragma unroll
+        for (int c = 0; c < 6; ++c) {
+          const int col = tn * kN + 192 * half + 32 * c;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (elect_one()) bulk_wait_group_read0();
+            __syncwarp();
+            if ((lane >> 4) == hh) {
+              const uint32_t rl = static_cast<uint32_t>(lane & 15);
+              const uint32_t dst = stg + rl * 64u;
+#pragma unroll
+              for (uint32_t q = 0; q < 4; ++q)
+                st_shared_v4(dst + 16u * (q ^ ((rl >> 1) & 3u)), yb[c].w[4 * q], yb[c].w[4 * q + 1],
+                             yb[c].w[4 * q + 2], yb[c].w[4 * q + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (elect_one()) {
+              tma_store_2d(&tm_y, stg, col, row0 + 16 * hh);
+              bulk_commit_group();
+            }
+            __syncwarp();
+          }
+        }
+        continue;
+      }
       uint32_t r[4][32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sp) << 16) + 128 * half;
 #pragma unroll
@@ -885,8 +1009,24 @@ static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 }
 
 size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
-template <bool kAct>
-size_t gemm_pair_smem_bytes() { return sizeof(PairSmem<kAct>) + 1024; }
+template <bool kAct, int kN>
+size_t gemm_pair_smem_bytes() { return sizeof(PairSmem<kAct, kN>) + 1024; }
+
+template <bool kAct, int kN>
+static bool pair_set_smem() {
+  return cudaFuncSetAttribute(gemm_dual_pair_kernel<kAct, kN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(gemm_pair_smem_bytes<kAct, kN>())) == cudaSuccess;
+}
+
+template <bool kAct, int kN>
+static int pair_clusters(cudaLaunchConfig_t cfg) {
+  cfg.dynamicSmemBytes = gemm_pair_smem_bytes<kAct, kN>();
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel<kAct, kN>, &cfg) != cudaSuccess)
+    return 0;
+  return n;
+}
 
 // Number of co-resident CTA pairs of the pair kernel on this device (0 if the
 // query fails); cached per device.
@@ -895,17 +1035,11 @@ static int pair_capacity() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] > 0) return cached[dev];
-  const size_t smem = gemm_pair_smem_bytes<false>();
-  const size_t smem_act = gemm_pair_smem_bytes<true>();
-  if (cudaFuncSetAttribute(gemm_dual_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess ||
-      cudaFuncSetAttribute(gemm_dual_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem_act)) != cudaSuccess)
+  if (!pair_set_smem<false, 256>() || !pair_set_smem<true, 256>() || !pair_set_smem<false, 384>())
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 148, 1, 1);
   cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -913,17 +1047,28 @@ static int pair_capacity() {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int n = 0;
-  int n2 = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_dual_pair_kernel<false>, &cfg) != cudaSuccess)
-    return 0;
-  cfg.dynamicSmemBytes = smem_act;
-  if (cudaOccupancyMaxActiveClusters(&n2, gemm_dual_pair_kernel<true>, &cfg) != cudaSuccess ||
-      n <= 0 || n2 <= 0)
-    return 0;
+  // one grid size serves every instantiation: the smallest co-resident count
+  int n = pair_clusters<false, 256>(cfg);
+  const int n2 = pair_clusters<true, 256>(cfg);
+  const int n3 = pair_clusters<false, 384>(cfg);
   if (n2 < n) n = n2;
+  if (n3 < n) n = n3;
+  if (n <= 0) return 0;
   cached[dev] = n;
   return n;
+}
+
+// Output columns per pair tile.  384 where it divides d_out and the epilogue
+// stores Y (a third fewer A bytes per FLOP and tile hand-offs); else 256.
+// W4A4_PAIR_TILE_N=256 in the environment keeps every launch on 256.
+static int pair_tile_n(int64_t d_out, bool act) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("W4A4_PAIR_TILE_N");
+    forced = (e != nullptr && strcmp(e, "256") == 0) ? 1 : 0;
+  }
+  if (act || forced == 1) return 256;
+  return d_out % 384 == 0 ? 384 : 256;
 }
 
 // Token counts up to this use the single-CTA kernel (a 256-row pair tile
@@ -935,7 +1080,9 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
                         void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act) {
   if (T == 0 || g.d_out == 0) return cudaSuccess;
   const bool pair = T >= kPairMinT && pair_capacity() > 0;
-  const uint32_t brows = pair ? 128 : BN;
+  const int tile_n = pair ? pair_tile_n(g.d_out, act != nullptr) : BN;
+  // B box rows: 256 (single CTA), 128 (pair, 256-wide tile), 64 (pair, 384-wide: 3 boxes)
+  const uint32_t brows = !pair ? BN : (tile_n == 384 ? 64 : 128);
   CUtensorMap tm_a, tm_b, tm_ao, tm_bo, tm_sfa, tm_sfb;
   memset(&tm_a, 0, sizeof(tm_a));
   memset(&tm_b, 0, sizeof(tm_b));
@@ -977,7 +1124,7 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   a.kt_j = static_cast<int>(g.kj_pad / 256);
   a.k_pad = static_cast<int>(g.k_pad);
   a.tiles_m = static_cast<int>((T + (pair ? 255 : BM - 1)) / (pair ? 256 : BM));
-  a.tiles_n = static_cast<int>((g.d_out + BN - 1) / BN);
+  a.tiles_n = static_cast<int>((g.d_out + tile_n - 1) / tile_n);
   a.act_inv_s = act ? act->inv_s : nullptr;
   a.act_aq = act ? act->aq : nullptr;
   a.act_sfa = act ? act->sfa : nullptr;
@@ -988,7 +1135,9 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   const int ntiles = a.tiles_m * a.tiles_n;
   if (pair) {
     const int npairs = ntiles < pair_capacity() ? ntiles : pair_capacity();
-    const size_t smem = act ? gemm_pair_smem_bytes<true>() : gemm_pair_smem_bytes<false>();
+    const size_t smem = act ? gemm_pair_smem_bytes<true, 256>()
+                            : (tile_n == 384 ? gemm_pair_smem_bytes<false, 384>()
+                                             : gemm_pair_smem_bytes<false, 256>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * npairs, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
@@ -1011,14 +1160,17 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
                      static_cast<uint64_t>(act->nblk) * 16, T, static_cast<uint64_t>(act->nblk) * 16,
                      32, 64, false, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true>, tm_a, tm_b, tm_ao, tm_bo,
+      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true, 256>, tm_a, tm_b, tm_ao, tm_bo,
                                 tm_sfa, tm_sfb, tm_y, a);
     }
     if (!make_tmap(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
                    static_cast<uint64_t>(ldy) * 2, 16, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false>, tm_a, tm_b, tm_ao, tm_bo, tm_sfa,
-                              tm_sfb, tm_y, a);
+    if (tile_n == 384)
+      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 384>, tm_a, tm_b, tm_ao, tm_bo,
+                                tm_sfa, tm_sfb, tm_y, a);
+    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 256>, tm_a, tm_b, tm_ao, tm_bo,
+                              tm_sfa, tm_sfb, tm_y, a);
   }
   const int sms = device_num_sms();
   const int grid = ntiles < sms ? ntiles : sms;

@@ -513,11 +513,12 @@ def run_gpu(args):
 def run_e2e(args, runs, w4, device, active):
     """Same step through the public calls with host buffers: every step copies
     X and W of each layer from pinned host memory, runs the whole path and
-    copies Y back.  The transfers of one layer overlap the work of the other:
-    host-to-device copies run on their own stream, in layer order; each
-    layer's compute waits only for its own inputs; each result copy waits only
-    for its own layer (PCIe is full duplex, so uploads and downloads also
-    overlap each other)."""
+    copies Y back, on three streams (uploads, compute, downloads; PCIe is
+    full duplex).  A layer's compute waits only for its own inputs and for
+    the previous step's download of its Y; its download waits only for its
+    compute; the next step's upload of its X and W waits only for this
+    step's compute of that layer to have read them.  So consecutive steps
+    pipeline: the uploads run back to back and set the pace."""
     import torch
     hosts = []
     for r in runs:
@@ -525,19 +526,23 @@ def run_e2e(args, runs, w4, device, active):
                       torch.empty(r.Y.shape, dtype=r.Y.dtype).pin_memory()))
     h2d = sum(x.numel() * 2 + w.numel() * 2 for x, w, _ in hosts)
     d2h = sum(y.numel() * 2 for _, _, y in hosts)
-    steps = max(1, min(args.steps, 3))
+    steps = max(3, min(args.steps, 8))
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    prev_c = [None] * len(runs)     # per layer: the previous step's compute is done
+    prev_o = [None] * len(runs)     # per layer: the previous step's download is done
 
     def step():
-        done_out = []
-        for r, (xh, wh, yh) in zip(runs, hosts):
-            # the previous step's result copy of this layer must have read Y
+        for i, (r, (xh, wh, yh)) in enumerate(zip(runs, hosts)):
+            if prev_c[i] is not None:
+                s_in.wait_event(prev_c[i])          # X and W are no longer read
             with torch.cuda.stream(s_in):
                 r.X.copy_(xh, non_blocking=True)
                 r.W.copy_(wh, non_blocking=True)
                 e_in = torch.cuda.Event()
                 e_in.record(s_in)
             s_comp.wait_event(e_in)
+            if prev_o[i] is not None:
+                s_comp.wait_event(prev_o[i])        # Y has been read out
             with torch.cuda.stream(s_comp):
                 r.offline()
                 r.online()
@@ -548,16 +553,15 @@ def run_e2e(args, runs, w4, device, active):
                 yh.copy_(r.Y, non_blocking=True)
                 e_o = torch.cuda.Event()
                 e_o.record(s_out)
-            done_out.append(e_o)
-        # a step ends when every result is on the host; the next step's uploads
-        # overwrite X and W, which this step's compute has finished with
-        for e in done_out:
-            s_in.wait_event(e)
-        e_end = torch.cuda.Event()
-        e_end.record(s_comp)
-        s_in.wait_event(e_end)
+            prev_c[i], prev_o[i] = e_c, e_o
+
+    def join():
+        # every step's results are on the host
+        s_in.wait_stream(s_comp)
+        s_in.wait_stream(s_out)
 
     step()
+    join()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -565,6 +569,7 @@ def run_e2e(args, runs, w4, device, active):
     t0.record(s_in)
     for _ in range(steps):
         step()
+    join()
     t1.record(s_in)
     torch.cuda.synchronize()
     ms = dist_max(t0.elapsed_time(t1) / steps, active, device)
@@ -573,7 +578,10 @@ def run_e2e(args, runs, w4, device, active):
     return {"value": round(aggregate(flops, world, ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
             "ms_per_step": round(ms, 3), "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "overlap": "uploads, compute and downloads on three streams, layers pipelined"}
+            "h2d_gbs": round(h2d / (ms * 1e-3) / 1e9, 1),
+            "overlap": "uploads, compute and downloads on three streams; consecutive steps "
+                       "pipelined (the timed region runs from the first upload to the last "
+                       "download)"}
 
 
 # ---------------------------------------------------------------------------

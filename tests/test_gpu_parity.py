@@ -278,6 +278,38 @@ def test_linear_parity_sampled_rows(L):
     gu.check_tolerance(gu.to_np_f32(Y)[rows].astype(np.float64), Y_ref, L.name)
 
 
+_TILE256_CHILD = """
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+from tests import test_gpu_parity as t
+for i, L in enumerate(t.TILE384):
+    X, W, pw = t._calibrate(L)
+    Y = t._linear(X, pw, L.T, L.d_out)
+    np.save(sys.argv[2] + f"/y{i}.npy", Y.view(torch.int16).cpu().numpy())
+"""
+
+
+def test_tile_widths_give_the_same_bits(tmp_path):
+    """The 256 x 384 pair tile against the 256 x 256 one on the same inputs:
+    W4A4_PAIR_TILE_N=256 is read once per process, so the 256-wide results
+    come from a child process."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, W4A4_PAIR_TILE_N="256")
+    r = subprocess.run([sys.executable, "-c", _TILE256_CHILD, root, str(tmp_path)], env=env,
+                       cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    for i, L in enumerate(TILE384):
+        X, W, pw = _calibrate(L)
+        Y = _linear(X, pw, L.T, L.d_out)
+        y256 = np.load(tmp_path / f"y{i}.npy")
+        assert np.array_equal(Y.view(torch.int16).cpu().numpy(), y256), L.name
+
+
 def test_gemm_matches_linear_and_is_deterministic():
     L = RAGGED
     X, W, pw = _calibrate(L)

@@ -88,6 +88,12 @@ FFN_CASES = [
     (100, 256, 640, 4, 32, 2),       # single-CTA GEMM (T <= 128), 128x1 stripes
     (520, 1024, 2048, 16, 0, 1),     # no outliers in the down layer, 32x32 tiles
     (300, 512, 1376, 8, 19, 1),      # 32x32 tiles with a non-trivial channel order
+    # d_ff a multiple of 384: the unfused path's up GEMM runs on 256 x 384
+    # pair tiles, the fused one on 256 x 256 (the two must agree bit for bit)
+    (300, 512, 1536, 8, 19, 0),      # outliers of the down layer in the last tile's half 1
+    (520, 1024, 768, 16, 0, 1),      # no outliers in the down layer, 32x32 tiles
+    (257, 256, 1152, 4, 64, 2),      # ragged M tile, 128x1 stripes
+    (300, 512, 768, 8, 300, 0),      # down layer with 16 MX blocks: whole code groups past it
 ]
 
 

@@ -99,6 +99,17 @@ def _ffn_cases(n=24, seed=77):
         layout = int(rng.integers(0, 3))
         out.append((f"ffn{i}_T{T}_{d_model}x{d_ff}_k{k_up}_{k_down}_l{layout}", T, d_model, d_ff,
                     k_up, k_down, layout, 100 + i))
+    # d_ff a multiple of 384 with T > 128: the unfused up GEMM on 384-wide
+    # tiles against the fused one on 256-wide tiles
+    for i in range(8):
+        T = int(rng.choice([129, 200, 333, 600]))
+        d_model = int(rng.integers(2, 65)) * 16
+        d_ff = int(rng.integers(1, 5)) * 384
+        k_up = int(min(d_model, rng.choice([0, 4, 16, 40])))
+        k_down = int(min(d_ff, rng.choice([0, 7, 19, 64, 300, d_ff])))
+        layout = int(rng.integers(0, 3))
+        out.append((f"ffn384_{i}_T{T}_{d_model}x{d_ff}_k{k_up}_{k_down}_l{layout}", T, d_model,
+                    d_ff, k_up, k_down, layout, 200 + i))
     return out
 
 

@@ -271,9 +271,9 @@ class ClockSampler:
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
-    "sha256": "d22c666630c87ef5a0a7612f6398c7c9b8cae53e6ad83c7e0ad292eb189538f5",
+    "sha256": "fdf6e8cbb15fd461000b350611761f06b41b430cae5d957ab8fb42b8306a63e9",
     "workload": "full",
-    "bytes_per_launch": (737091840 + 1560132352 + 1584012800 + 572660736) / 2,
+    "bytes_per_launch": (581736448 + 1551764992 + 1417102080 + 573487104) / 2,
 }
 
 

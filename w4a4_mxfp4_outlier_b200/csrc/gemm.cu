@@ -61,6 +61,7 @@ constexpr int TMEM_SFA_COL = 256;             // 2 atoms x 4 columns
 constexpr int TMEM_SFB_COL = 264;             // 2 atoms x 8 columns
 constexpr int TMEM_SF_BUF = 32;               // scale buffers alternate by K tile: +0 / +32 columns
 constexpr int GROUP_M = 16;                   // tile raster: 16 M tiles per sweep of N
+constexpr int GROUP_M_384 = 24;               // the same for 384-wide pair tiles (measured best)
 
 struct GemmSmem {
   uint8_t stage[STAGES][STAGE_BYTES];         // 1024-aligned (each part 1024-aligned)
@@ -224,11 +225,14 @@ __device__ __forceinline__ void act_store_scales(const GemmArgs& a, int row, int
     *reinterpret_cast<uint32_t*>(a.act_sfa + sf_offset(row, b0, a.act_nblk)) = codes;
 }
 
+// Tile t of the raster: groups of kGroupM M tiles, each group swept N tile by
+// N tile, M fastest within the group.
+template <int kGroupM = GROUP_M>
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
-  const int per_group = GROUP_M * tiles_n;
+  const int per_group = kGroupM * tiles_n;
   const int g = t / per_group;
-  const int first_m = g * GROUP_M;
-  const int gm = tiles_m - first_m < GROUP_M ? tiles_m - first_m : GROUP_M;
+  const int first_m = g * kGroupM;
+  const int gm = tiles_m - first_m < kGroupM ? tiles_m - first_m : kGroupM;
   const int w = t - g * per_group;
   tn = w / gm;
   tm = first_m + w % gm;
@@ -607,7 +611,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint32_t it = 0, s = 0, ph = 0;
     for (int t = pair; t < ntiles && ok; t += npairs) {
       int tm, tn;
-      tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
+      tile_coords<kN == 384 ? GROUP_M_384 : GROUP_M>(t, args.tiles_m, args.tiles_n, tm, tn);
       const int m_rows = tm * 256 + 128 * static_cast<int>(rank);
       const int n_rows = tn * kN + 128 * static_cast<int>(rank);
       const int n_rows2 = tn * kN + 256 + 64 * static_cast<int>(rank);   // kN = 384 only
@@ -817,7 +821,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint32_t tcount = 0;
     for (int t = pair; t < ntiles; t += npairs, ++tcount) {
       int tm, tn;
-      tile_coords(t, args.tiles_m, args.tiles_n, tm, tn);
+      tile_coords<kN == 384 ? GROUP_M_384 : GROUP_M>(t, args.tiles_m, args.tiles_n, tm, tn);
       int ready = 0;
       if (lane == 0)
         ready = mbar_wait_bounded(&sm.acc_full, tcount & 1u, abort_flag, DEVERR_TIMEOUT_EPILOGUE);

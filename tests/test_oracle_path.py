@@ -60,6 +60,12 @@ def test_smoothing_closed_forms():
     # alpha = 0.7, a = 2^10, w = 2^-10 -> s = 2^7 * 2^3 = 2^10
     s, _ = orc.smoothing_factors(np.array([1024.0], np.float32), np.array([2.0**-10], np.float32), 0.7)
     assert abs(float(s[0]) - 1024.0) <= 1024.0 * 2**-22
+    # the activation magnitude carries exponent alpha, the weight's 1 - alpha
+    # (review sec. 3.2, eq. s_j): alpha = 0.7, a = 2^10, w = 1 -> s = 2^7;
+    # a = 1, w = 2^10 -> s = 2^-3 (exchanged exponents would give 2^3, 2^-7)
+    s, _ = orc.smoothing_factors(np.array([1024.0, 1.0], np.float32),
+                                 np.array([1.0, 1024.0], np.float32), 0.7)
+    np.testing.assert_allclose(s.astype(np.float64), [128.0, 0.125], rtol=2**-22)
     # zero magnitudes are clamped at 1e-5: a = 0, w = 0, alpha = 0.5 -> s = 1e-5^0.5 / 1e-5^0.5 = 1
     s, _ = orc.smoothing_factors(np.zeros(1, np.float32), np.zeros(1, np.float32), 0.5)
     assert s[0] == 1.0

@@ -18,7 +18,8 @@ _orig = {name: getattr(orc, name) for name in (
     "e2m1_codes", "mx_shared_exponent", "pack_nibbles", "unpack_nibbles",
     "smoothing_factors", "outlier_scores", "select_outliers", "fold_weight",
     "dual_branch_product", "pack_weight", "f32_to_bf16_bits", "gelu_bf16",
-    "col_absmax")}
+    "col_absmax", "dequant_mxfp4", "prep_activation", "calibrate",
+    "mxfp4_quantize_blocks")}
 
 
 def _e2m1_ties_away(q):
@@ -119,7 +120,105 @@ def _absmax_signed(A, running=None):
     return m.astype(np.float32)
 
 
+def _e2m1_toward_zero(q):
+    """Magnitudes rounded down onto the grid instead of to the nearest."""
+    a = np.minimum(np.abs(np.asarray(q, dtype=np.float64)), orc.E2M1_GRID[-1])
+    pick = np.sum(a[..., None] >= orc.E2M1_GRID, axis=-1) - 1
+    sign = np.signbit(np.asarray(q, dtype=np.float32)).astype(np.int64)
+    return (pick | (sign << 3)).astype(np.uint8)
+
+
+def _e2m1_saturate_at_4(q):
+    """Saturation at 4 (the grid's 6 never produced)."""
+    c = _orig["e2m1_codes"](q)
+    return np.where((c & 7) == 7, c - 1, c).astype(np.uint8)
+
+
+def _exponent_ceil(amax):
+    """ceil(log2 amax) - 2 instead of floor."""
+    a = np.asarray(amax, dtype=np.float64)
+    m, ex = np.frexp(a)
+    e = ex.astype(np.int64) - 1 - orc.E2M1_EMAX + (m != 0.5).astype(np.int64)
+    e = np.where(a == 0.0, -orc.E8M0_BIAS, e)
+    return np.clip(e, -127, 127)
+
+
+def _dequant_bias_126(packed, sf, ncols=None):
+    """E8M0 read with bias 126."""
+    return _orig["dequant_mxfp4"](packed, sf.astype(np.int64) + 1, ncols)
+
+
+def _topk_smallest(score, k):
+    """The k smallest scores taken as outliers."""
+    d = score.shape[0]
+    order = np.lexsort((np.arange(d), score.astype(np.float64)))
+    return np.sort(order[:k]).astype(np.int32), np.sort(order[k:]).astype(np.int32)
+
+
+def _topk_unsorted(score, k):
+    """O left in score order instead of ascending."""
+    d = score.shape[0]
+    order = np.lexsort((np.arange(d), -score.astype(np.float64)))
+    return order[:k].astype(np.int32), np.sort(order[k:]).astype(np.int32)
+
+
+def _xo_unsmoothed(X, inv_s, O, J, row_chunk=512):
+    """The outlier columns taken from X before smoothing."""
+    out = _orig["prep_activation"](X, inv_s, O, J, row_chunk)
+    out["xo"] = orc.f32_to_bf16_bits(X[:, O].astype(np.float32))
+    return out
+
+
+def _w_hp_unfolded(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
+    """The outlier weight rows left unfolded (s not applied)."""
+    out = _orig["pack_weight"](W, s, O, J, layout, row_chunk)
+    out["w_hp"] = orc.f32_to_bf16_bits(W[:, O].astype(np.float32))
+    return out
+
+
+def _stripes_as_blocks(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
+    """128x1 stripes packed with one scale per 32x1 block."""
+    if layout == orc.LAYOUT_128x1:
+        layout = orc.LAYOUT_32x1
+    return _orig["pack_weight"](W, s, O, J, layout, row_chunk)
+
+
+def _absmax_ignores_running(A, running=None):
+    """Calibration over several batches keeps only the last batch."""
+    return _orig["col_absmax"](A, None)
+
+
+def _calibrate_first_batch(X_batches, W, alpha, k):
+    """Outlier scores from the first calibration batch only."""
+    c = _orig["calibrate"](X_batches, W, alpha, k)
+    if not isinstance(X_batches, np.ndarray) and len(X_batches) > 1:
+        score = orc.outlier_scores(X_batches[0], c["inv_s"])
+        O, J = orc.select_outliers(score, k)
+        c = {**c, "score": score, "O": O, "J": J}
+    return c
+
+
+def _block_amax_signed(V, block_amax=None):
+    """Block scale from the largest value rather than the largest magnitude."""
+    if block_amax is None:
+        block_amax = np.max(np.asarray(V, dtype=np.float32), axis=-1)
+        block_amax = np.maximum(block_amax, 0.0)
+    return _orig["mxfp4_quantize_blocks"](V, block_amax)
+
+
 MUTANTS = {
+    "e2m1_toward_zero": {"e2m1_codes": _e2m1_toward_zero},
+    "e2m1_saturate_at_4": {"e2m1_codes": _e2m1_saturate_at_4},
+    "exponent_ceil": {"mx_shared_exponent": _exponent_ceil},
+    "dequant_bias_126": {"dequant_mxfp4": _dequant_bias_126},
+    "topk_smallest": {"select_outliers": _topk_smallest},
+    "topk_unsorted": {"select_outliers": _topk_unsorted},
+    "xo_unsmoothed": {"prep_activation": _xo_unsmoothed},
+    "w_hp_unfolded": {"pack_weight": _w_hp_unfolded},
+    "stripes_as_blocks": {"pack_weight": _stripes_as_blocks},
+    "absmax_ignores_running": {"col_absmax": _absmax_ignores_running},
+    "calibrate_first_batch": {"calibrate": _calibrate_first_batch},
+    "block_amax_signed": {"mxfp4_quantize_blocks": _block_amax_signed},
     "e2m1_ties_away": {"e2m1_codes": _e2m1_ties_away},
     "e2m1_unsigned_zero": {"e2m1_codes": _e2m1_unsigned_zero},
     "exponent_minus_1": {"mx_shared_exponent": _exponent_minus_1},

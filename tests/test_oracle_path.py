@@ -83,6 +83,22 @@ def test_smoothing_balances_ranges_at_half():
     np.testing.assert_allclose(xs, np.sqrt(act.astype(np.float64) * wsc), rtol=1e-6)
 
 
+def test_calibration_over_batches_equals_their_concatenation():
+    """Calibrating on several batches is calibrating on their union: each
+    per-channel magnitude is a max over every calibration token (review
+    sec. 3.2, magnitudes collected over the calibration data, which the
+    pipeline gathers in batches across timesteps)."""
+    X, W = _small(T=192, d_in=96, n_out=0)
+    X1, X2, X3 = X[:64].copy(), X[64:128].copy(), X[128:].copy()
+    X2[:, 5] *= 64.0           # an outlier channel seen only in the second batch
+    X3[:, 70] *= 128.0         # and one seen only in the third (powers of 2: exact)
+    full = orc.calibrate(np.vstack([X1, X2, X3]), W, 0.6, 4)
+    parts = orc.calibrate([X1, X2, X3], W, 0.6, 4)
+    for key in ("act_scale", "w_scale", "s", "inv_s", "score", "O", "J"):
+        np.testing.assert_array_equal(parts[key], full[key], err_msg=key)
+    assert {5, 70} <= set(full["O"].tolist())
+
+
 def test_score_equals_scaled_act_scale():
     """max_t fl32(|x| * inv_s) = fl32(max_t |x| * inv_s): rounding is monotone,
     so the score needs no second pass over X."""

@@ -11,8 +11,7 @@ tensor core would read the scales elsewhere and Y would differ).
 import os
 import subprocess
 import sys
-
-import pytest
+from concurrent.futures import ThreadPoolExecutor
 
 from tests import oracle_mutants
 
@@ -32,10 +31,15 @@ def test_pins_pass_with_nothing_planted():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
-@pytest.mark.parametrize("mutant", sorted(oracle_mutants.MUTANTS))
-def test_pins_catch_planted_mistake(mutant):
-    r = _run_pins(mutant)
-    # 1 = tests failed (an exception in a test also counts as a failure);
-    # anything else would mean the harness itself broke
-    assert r.returncode == 1, f"{mutant}: pins passed or the run broke (rc {r.returncode})\n" + \
-        r.stdout[-3000:]
+def test_pins_catch_every_planted_mistake():
+    # one child per mutant, several at a time (each spends most of its few
+    # seconds importing); exit code 1 = tests failed (an exception in a test
+    # counts as a failure), anything else would mean the harness broke
+    names = sorted(oracle_mutants.MUTANTS)
+    workers = max(2, min(8, os.cpu_count() or 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        results = dict(zip(names, ex.map(_run_pins, names)))
+    missed = {n: r.returncode for n, r in results.items() if r.returncode != 1}
+    assert not missed, "pins passed or the run broke: " + ", ".join(
+        f"{n} (rc {rc})" for n, rc in missed.items()) + "\n" + \
+        "\n".join(results[n].stdout[-1500:] for n in missed)

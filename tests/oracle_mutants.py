@@ -19,7 +19,7 @@ _orig = {name: getattr(orc, name) for name in (
     "smoothing_factors", "outlier_scores", "select_outliers", "fold_weight",
     "dual_branch_product", "pack_weight", "f32_to_bf16_bits", "gelu_bf16",
     "col_absmax", "dequant_mxfp4", "prep_activation", "calibrate",
-    "mxfp4_quantize_blocks")}
+    "mxfp4_quantize_blocks", "_pad_cols", "smooth_activation")}
 
 
 def _e2m1_ties_away(q):
@@ -206,7 +206,50 @@ def _block_amax_signed(V, block_amax=None):
     return _orig["mxfp4_quantize_blocks"](V, block_amax)
 
 
+def _pad_repeat_last(A, ncols):
+    """The last partial block completed with copies of its last column."""
+    if A.shape[1] == ncols or A.shape[1] == 0:
+        return _orig["_pad_cols"](A, ncols)
+    out = np.empty((A.shape[0], ncols), dtype=A.dtype)
+    out[:, :A.shape[1]] = A
+    out[:, A.shape[1]:] = A[:, -1:]
+    return out
+
+
+def _smooth_f64(X, inv_s):
+    """The smoothing product taken in float64 and never rounded to float32
+    (with _quantize_f64: the whole encode done in float64)."""
+    return X.astype(np.float64) * inv_s.astype(np.float64)[None, :]
+
+
+def _quantize_f64(V, block_amax=None):
+    V = np.asarray(V, dtype=np.float64)
+    if block_amax is None:
+        block_amax = np.max(np.abs(V), axis=-1)
+    e = orc.mx_shared_exponent(block_amax)
+    q = np.ldexp(V, (-e)[..., None].astype(np.int32))
+    return (e + orc.E8M0_BIAS).astype(np.uint8), orc.e2m1_codes(q)
+
+
+def _fold_rounded_bf16(W, s):
+    """The folded weight rounded to bf16 before it is quantised."""
+    return orc.bf16_bits_to_f32(orc.f32_to_bf16_bits((W * s[None, :]).astype(np.float32)))
+
+
+def _dequant_tiled_scales(packed, sf, ncols=None):
+    """Scales spread over the row with tile (s0 s1 .. s0 s1 ..) instead of repeat."""
+    codes = orc.unpack_nibbles(packed)
+    K = codes.shape[-1]
+    scale = np.ldexp(1.0, sf.astype(np.int64) - orc.E8M0_BIAS)
+    vals = orc.e2m1_value(codes) * np.tile(scale, (1,) * (scale.ndim - 1) + (orc.MX_BLOCK,))[..., :K]
+    return vals if ncols is None else vals[..., :ncols]
+
+
 MUTANTS = {
+    "pad_repeat_last": {"_pad_cols": _pad_repeat_last},
+    "encode_in_f64": {"smooth_activation": _smooth_f64, "mxfp4_quantize_blocks": _quantize_f64},
+    "fold_rounded_bf16": {"fold_weight": _fold_rounded_bf16},
+    "dequant_tiled_scales": {"dequant_mxfp4": _dequant_tiled_scales},
     "e2m1_toward_zero": {"e2m1_codes": _e2m1_toward_zero},
     "e2m1_saturate_at_4": {"e2m1_codes": _e2m1_saturate_at_4},
     "exponent_ceil": {"mx_shared_exponent": _exponent_ceil},

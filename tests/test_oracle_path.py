@@ -99,6 +99,27 @@ def test_calibration_over_batches_equals_their_concatenation():
     assert {5, 70} <= set(full["O"].tolist())
 
 
+def test_smoothing_product_is_one_float32_multiply():
+    """x * inv_s is rounded to float32 before it is encoded (the reading of
+    review sec. 3.2's "divide by s": one IEEE float32 multiply by fl32(1/s)).
+    Hand-worked: x = 0.25390625 (bf16), inv_s = 0.98461538553237915 (float32);
+    the exact product is 0.25 + 2.3e-10, its float32 rounding exactly 0.25.
+    With 4.0 in the same block (scale 2^0), 0.25 is the tie between the E2M1
+    codes for 0 and 0.5 and goes to the even one, 0; the unrounded product
+    would encode as 0.5."""
+    x = np.float32(0.25390625)
+    inv = np.float32(0.98461538553237915)
+    assert np.float32(x * inv) == np.float32(0.25)
+    assert float(x) * float(inv) > 0.25
+    X = np.zeros((1, 32), np.float32)
+    X[0, 0], X[0, 1] = x, 4.0
+    inv_s = np.ones(32, np.float32)
+    inv_s[0] = inv
+    out = orc.prep_activation(X, inv_s, np.zeros(0, np.int32), np.arange(32, dtype=np.int32))
+    assert out["sfa"][0, 0] == 127                      # shared exponent 0
+    assert out["aq"][0, 0] == 0x60                      # codes 0 (x) and 6 (4.0)
+
+
 def test_score_equals_scaled_act_scale():
     """max_t fl32(|x| * inv_s) = fl32(max_t |x| * inv_s): rounding is monotone,
     so the score needs no second pass over X."""

@@ -245,7 +245,49 @@ def _dequant_tiled_scales(packed, sf, ncols=None):
     return vals if ncols is None else vals[..., :ncols]
 
 
+def _gelu_double_round(y):
+    """tanh-form GELU evaluated in float32, then rounded to bf16 (two roundings)."""
+    yv = np.asarray(y, dtype=np.float32)
+    c = np.float32(np.sqrt(2.0 / np.pi))
+    g = np.float32(0.5) * yv * (np.float32(1.0) + np.tanh(c * (yv + np.float32(0.044715) * yv ** 3)))
+    return orc.f32_to_bf16_bits(g.astype(np.float32))
+
+
+def _no_scale_floor(act_scale, w_scale, alpha):
+    """Zero magnitudes not clamped (s = 0^a / 0^b)."""
+    a = act_scale.astype(np.float64)
+    w = w_scale.astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s64 = np.power(a, float(alpha)) / np.power(w, 1.0 - float(alpha))
+        s = s64.astype(np.float32)
+        inv_s = (1.0 / s.astype(np.float64)).astype(np.float32)
+    return s, inv_s
+
+
+def _stripes_offset(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
+    """128x1 stripes starting at the second MX block instead of the first."""
+    if layout != orc.LAYOUT_128x1:
+        return _orig["pack_weight"](W, s, O, J, layout, row_chunk)
+    out = _orig["pack_weight"](W, s, O, J, orc.LAYOUT_32x1, row_chunk)
+    nb = out["sfb"].shape[1]
+    Wf = orc.fold_weight(W.astype(np.float32), s.astype(np.float32)).astype(np.float32)
+    WJ = orc._pad_cols(Wf[:, J], nb * orc.MX_BLOCK).reshape(W.shape[0], nb, orc.MX_BLOCK)
+    amax = np.max(np.abs(WJ), axis=-1)
+    grp = (np.arange(nb) + 1) // 4
+    stripe = np.zeros_like(amax)
+    for g_ in np.unique(grp):
+        cols = grp == g_
+        stripe[:, cols] = amax[:, cols].max(axis=1, keepdims=True)
+    sc, codes = orc.mxfp4_quantize_blocks(WJ, stripe)
+    out["sfb"] = sc
+    out["wq"] = orc.pack_nibbles(codes.reshape(W.shape[0], nb * orc.MX_BLOCK))
+    return out
+
+
 MUTANTS = {
+    "gelu_double_round": {"gelu_bf16": _gelu_double_round},
+    "no_scale_floor": {"smoothing_factors": _no_scale_floor},
+    "stripes_offset": {"pack_weight": _stripes_offset},
     "pad_repeat_last": {"_pad_cols": _pad_repeat_last},
     "encode_in_f64": {"smooth_activation": _smooth_f64, "mxfp4_quantize_blocks": _quantize_f64},
     "fold_rounded_bf16": {"fold_weight": _fold_rounded_bf16},

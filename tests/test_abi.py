@@ -94,6 +94,46 @@ def test_calls_validate_before_launch():
     assert w4._gemm_dual(None, None, None, 0, ctypes.byref(pw), None, 32, None) == w4.OK
 
 
+def test_ffn_calls_validate_before_launch():
+    # Pointers here are never dereferenced: every call returns before any CUDA work.
+    f = 0x1000
+    pw = _raw_pw()                                  # 64 -> 32, k = 4
+    nxt = _raw_pw(d_in=32, d_out=64, k=4, fake=0x2000)
+    # GELU: row strides below the width, missing buffers, negative T; empty is a no-op
+    assert w4._gelu_bf16(f, 8, 64, 63, f, 64, None) == w4.ERR_INVALID_ARG
+    assert w4._gelu_bf16(f, 8, 64, 64, f, 63, None) == w4.ERR_INVALID_ARG
+    assert w4._gelu_bf16(None, 8, 64, 64, f, 64, None) == w4.ERR_INVALID_ARG
+    assert w4._gelu_bf16(f, -1, 64, 64, f, 64, None) == w4.ERR_INVALID_ARG
+    assert w4._gelu_bf16(None, 0, 64, 64, None, 64, None) == w4.OK
+    # channel order of the next layer: a valid packed layer and both outputs
+    assert w4._ffn_link(None, f, f, None) == w4.ERR_INVALID_ARG
+    assert w4._ffn_link(ctypes.byref(nxt), None, f, None) == w4.ERR_INVALID_ARG
+    assert w4._ffn_link(ctypes.byref(_raw_pw(layout=7)), f, f, None) == w4.ERR_INVALID_ARG
+    # packing permuted rows: the same checks as the plain pack, plus the row map
+    assert w4._pack_weight_rows(f, 63, f, f, ctypes.byref(pw), None) == w4.ERR_INVALID_ARG
+    assert w4._pack_weight_rows(f, 68, f, f, ctypes.byref(pw), None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._pack_weight_rows(f + 2, 64, f, f, ctypes.byref(pw), None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._pack_weight_rows(f, 64, f, None, ctypes.byref(pw), None) == w4.ERR_INVALID_ARG
+    # permuting a packed layer: same shape and layout, a row map, never in place
+    other = _raw_pw(fake=0x3000)
+    assert w4._permute_packed_rows(ctypes.byref(pw), f, ctypes.byref(_raw_pw(d_out=48, fake=0x3000)),
+                                   None) == w4.ERR_INVALID_ARG
+    assert w4._permute_packed_rows(ctypes.byref(pw), f, ctypes.byref(_raw_pw(layout=1, fake=0x3000)),
+                                   None) == w4.ERR_INVALID_ARG
+    assert w4._permute_packed_rows(ctypes.byref(pw), None, ctypes.byref(other), None) == w4.ERR_INVALID_ARG
+    assert w4._permute_packed_rows(ctypes.byref(pw), f, ctypes.byref(_raw_pw()), None) == w4.ERR_INVALID_ARG
+    # the fused epilogue: the next layer's d_in is this layer's d_out, its
+    # column order's inv_s is given, its buffers are there and 16-byte aligned
+    act = lambda T=8, nx=nxt, inv=f, aqn=f + 0x100: w4._gemm_dual_act(
+        f, f, f, T, ctypes.byref(pw), ctypes.byref(nx), inv, aqn, f + 0x200, f + 0x300, None)
+    assert act(nx=_raw_pw(d_in=48, d_out=64, fake=0x2000)) == w4.ERR_INVALID_ARG
+    assert act(inv=None) == w4.ERR_INVALID_ARG
+    assert act(T=-1) == w4.ERR_INVALID_ARG
+    assert act(aqn=None) == w4.ERR_INVALID_ARG
+    assert act(aqn=f + 0x101) == w4.ERR_UNSUPPORTED_SHAPE
+    assert act(T=0) == w4.OK
+
+
 def test_calib_validation():
     assert w4._calib_observe(0x1000, 4, 8, 4, 0x1000, 1, None) == w4.ERR_INVALID_ARG      # lda < cols
     assert w4._calib_observe(0x1000, 4, 12, 12, 0x1000, 1, None) == w4.ERR_UNSUPPORTED_SHAPE

@@ -134,6 +134,33 @@ def test_ffn_calls_validate_before_launch():
     assert act(T=0) == w4.OK
 
 
+def test_pack_host_and_metric_calls_validate_before_launch():
+    # Pointers here are never dereferenced: every call returns before any CUDA work.
+    f = 0x1000
+    pw = _raw_pw()                                  # 64 -> 32, k = 4
+    # weight pack: row stride, alignment, missing W or s, a malformed record
+    assert w4._pack_weight(f, 63, f, ctypes.byref(pw), None) == w4.ERR_INVALID_ARG
+    assert w4._pack_weight(f, 68, f, ctypes.byref(pw), None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._pack_weight(f + 8, 64, f, ctypes.byref(pw), None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._pack_weight(None, 64, f, ctypes.byref(pw), None) == w4.ERR_INVALID_ARG
+    assert w4._pack_weight(f, 64, None, ctypes.byref(pw), None) == w4.ERR_INVALID_ARG
+    no_inv = _raw_pw()
+    no_inv.inv_s = None
+    assert w4._pack_weight(f, 64, f, ctypes.byref(no_inv), None) == w4.ERR_INVALID_ARG
+    # the host-buffer layer: every buffer, a big enough workspace; T = 0 is a no-op
+    ws = w4.workspace_size(8, 64, 32, 4)
+    assert w4._linear_host(f, -1, ctypes.byref(pw), f, f, ws, f, f, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_host(None, 8, ctypes.byref(pw), f, f, ws, f, f, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_host(f, 8, ctypes.byref(pw), f, f, ws, f, None, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_host(f, 8, ctypes.byref(pw), f, f, ws - 1, f, f, None) == w4.ERR_INVALID_ARG
+    assert w4._linear_host(f, 0, ctypes.byref(pw), None, None, 0, None, None, None) == w4.OK
+    # the error-sum reduction used by the layer search
+    assert w4._error_sums(f, 31, f, 32, 8, 32, f, None) == w4.ERR_INVALID_ARG
+    assert w4._error_sums(f, 32, f, 31, 8, 32, f, None) == w4.ERR_INVALID_ARG
+    assert w4._error_sums(f, 32, f, 32, 8, 32, None, None) == w4.ERR_INVALID_ARG
+    assert w4._error_sums(None, 32, f, 32, 8, 32, f, None) == w4.ERR_INVALID_ARG
+
+
 def test_calib_validation():
     assert w4._calib_observe(0x1000, 4, 8, 4, 0x1000, 1, None) == w4.ERR_INVALID_ARG      # lda < cols
     assert w4._calib_observe(0x1000, 4, 12, 12, 0x1000, 1, None) == w4.ERR_UNSUPPORTED_SHAPE

@@ -1,20 +1,26 @@
 """Benchmark of the W4A4 dual-branch linear on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full|ffn0|ffn2|tiny|sweep]
-                    [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload full|full_up|full_down|mid_up|mid_down|ffn0|ffn2|tiny|sweep
+                                |ffn|ffn_mid]
 
 One step is one pass of the whole path over one batch of synthetic input,
 for every layer of the workload: calibration absmax of X and of W, the
 finalisation (s, score, top-k), the weight pack, the activation prep and the
 dual-branch GEMM -- all through the C-ABI of libw4a4.  The default workload
-is the 720x1280x61 token count (T = 57600) through the FFN up-projection
-(5120 -> 13824, k = 32) and then the down-projection (13824 -> 5120, k = 64).
+is T = 57600 tokens (16 x 45 x 80 latent positions) on the FFN up-projection
+shape (5120 -> 13824, k = 32) and on the down-projection shape (13824 ->
+5120, k = 64), each layer with its own synthetic input.  The ffn workloads
+instead time the online FFN forward with the fused epilogue.
 
 ``value`` is whole-step effective TFLOPS, 2 T d_in d_out summed over the
 layers divided by the step time (outlier columns counted at the 4-bit
 rate).  Per-kernel numbers come from CUDA events recorded on the launching
-stream around each launch inside the timed region.  Inputs are larger than
-L2 (X is 590 MB / 1.59 GB), so no flush is needed between steps.
+stream around each launch inside the timed region.  The full workload's
+inputs are larger than L2 (X is 590 MB / 1.59 GB), so nothing is flushed;
+where a step's inputs are under twice the L2 size a 256 MB buffer is written
+between steps, outside each step's own events.  ``e2e`` repeats the step
+from pinned host buffers with the copies inside the timed region.
 
 Under torchrun each rank runs the same per-GPU workload on its own token
 shard (weak scaling, no collective on the data path); the step time is the

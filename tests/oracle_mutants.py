@@ -284,7 +284,28 @@ def _stripes_offset(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
     return out
 
 
+def _prep_zero_in_place(X, inv_s, O, J, row_chunk=512):
+    """O columns zeroed in place and the MX blocks formed over all d_in
+    columns, instead of over the compacted J positions."""
+    Xz = np.array(X, dtype=np.float32, copy=True)
+    Xz[:, O] = 0.0
+    out = _orig["prep_activation"](Xz, inv_s, np.zeros(0, np.int32),
+                                   np.arange(X.shape[1], dtype=np.int32), row_chunk)
+    out["xo"] = _orig["prep_activation"](X, inv_s, O, J, row_chunk)["xo"]
+    return out
+
+
+def _pack_zero_in_place(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
+    Wz = np.array(W, dtype=np.float32, copy=True)
+    Wz[:, O] = 0.0
+    out = _orig["pack_weight"](Wz, s, np.zeros(0, np.int32), np.arange(W.shape[1], dtype=np.int32),
+                               layout, row_chunk)
+    out["w_hp"] = _orig["pack_weight"](W, s, O, J, layout, row_chunk)["w_hp"]
+    return out
+
+
 MUTANTS = {
+    "zero_in_place": {"prep_activation": _prep_zero_in_place, "pack_weight": _pack_zero_in_place},
     "gelu_double_round": {"gelu_bf16": _gelu_double_round},
     "no_scale_floor": {"smoothing_factors": _no_scale_floor},
     "stripes_offset": {"pack_weight": _stripes_offset},

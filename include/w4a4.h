@@ -22,7 +22,11 @@
  *    elements; W is [d_out, d_in] bf16 (row n = output channel n; this is the
  *    transpose of the pages' d_in x d_out W); Y is [T, d_out] bf16.
  *  - Arguments are validated before anything is launched.  On a non-OK
- *    return nothing was enqueued and outputs are untouched.
+ *    return nothing was enqueued and outputs are untouched.  Calls that
+ *    enqueue several steps (w4a4_linear, w4a4_linear_host,
+ *    w4a4_linear_noalloc, w4a4_gemm_dual_act) check the arguments of every
+ *    step, and build the GEMM's tensor maps, before the first one; only a
+ *    failing launch itself (W4A4_ERR_CUDA) can leave earlier steps enqueued.
  *  - Supported shapes: d_in % 8 == 0, d_out % 16 == 0, row strides % 8 == 0,
  *    all pointers 16-byte aligned, d_in <= 16384.
  *    Anything else returns W4A4_ERR_UNSUPPORTED_SHAPE.
@@ -320,9 +324,13 @@ w4a4_status w4a4_gemm_dual_act(const uint8_t* aq, const uint8_t* sfa, const void
  *   are never stored -- but calls whose GPU work overlaps (other streams,
  *   other host threads) race on the array and must be serialised by the
  *   caller.
- *   Set-up: the first call on each device looks up the array's device address
- *   (a host-side query, with that device current; nothing is allocated).
- *   Make that first call before any stream capture.
+ *   Set-up: the first call in each CUDA context looks up the array's device
+ *   address in that context (a host-side query with the device current;
+ *   nothing is allocated) -- normally once per device, in its primary
+ *   context.  The lookup is cached by the context's unique id, so a caller's
+ *   own driver-API context, or a new primary context after cudaDeviceReset,
+ *   gets its own address.  Make the first call in a context before any stream
+ *   capture.
  * Arguments, layouts and the other errors are those of w4a4_linear. */
 w4a4_status w4a4_linear_noalloc(const void* X, int64_t T, int64_t ldx,
                                 const w4a4_packed_weight* pw, void* Y, int64_t ldy,

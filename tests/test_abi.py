@@ -221,3 +221,34 @@ def test_packed_image_header_checks():
     sizes = [32 * d.kj_pad // 2, d.sfb_rows * d.nblk, 32 * d.k_pad * 2, 256, 256, 16, 240]
     assert n.value == 256 + sum(-(-x // 64) * 64 for x in sizes)
 
+
+
+def test_composite_calls_check_every_step_before_the_first_launch():
+    # Pointers here are never dereferenced: the output checks of the GEMM step
+    # reject these calls before the prep step (or the upload) is enqueued.
+    f = 0x1000
+    pw = _raw_pw()                                  # 64 -> 32, k = 4
+    ws = w4.workspace_size(8, 64, 32, 4)
+    # Y row stride not a multiple of 8 (ldy = 36 >= d_out = 32), Y misaligned
+    assert w4._linear(f, 8, 64, ctypes.byref(pw), f, ws, f, 36, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear(f, 8, 64, ctypes.byref(pw), f, ws, f + 8, 32, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear_noalloc(f, 8, 64, ctypes.byref(pw), f, 36, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear_noalloc(f, 8, 64, ctypes.byref(pw), f + 8, 32, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear_noalloc(f + 2, 8, 64, ctypes.byref(pw), f, 32, None) == w4.ERR_UNSUPPORTED_SHAPE
+    # the host-buffer layer: misaligned device buffers are caught before the upload
+    assert w4._linear_host(f, 8, ctypes.byref(pw), f + 8, f, ws, f, f, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear_host(f, 8, ctypes.byref(pw), f, f, ws, f + 8, f, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert w4._linear_host(f, 8, ctypes.byref(pw), f, f + 8, ws, f, f, None) == w4.ERR_UNSUPPORTED_SHAPE
+
+
+def test_binding_rejects_what_is_not_bf16_rows():
+    import torch
+    X = torch.zeros(8, 64, dtype=torch.bfloat16)
+    w4._rows_bf16(X, "x", cuda=False)                   # dense host rows pass
+    for bad in (X.t(), X.float(), X[:, ::2], X.reshape(-1)):
+        with pytest.raises(w4.W4A4Error) as e:
+            w4._rows_bf16(bad, "x", cuda=False)
+        assert e.value.status == w4.ERR_INVALID_ARG
+    with pytest.raises(w4.W4A4Error) as e:
+        w4._rows_bf16(X, "x")                           # host memory where device rows are read
+    assert e.value.status == w4.ERR_INVALID_ARG

@@ -122,6 +122,23 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
+def _rows_bf16(t: torch.Tensor, what: str, device=None, cuda: bool = True):
+    """The library reads a bf16 matrix as rows of contiguous elements with a
+    row stride: reject anything else (another dtype, a transposed or
+    column-strided view, a tensor on another device) before the call, since
+    the C ABI sees only a pointer and a row stride."""
+    ok = (t.dtype == torch.bfloat16 and t.dim() == 2 and (t.stride(1) == 1 or t.shape[1] <= 1)
+          and t.is_cuda == cuda and (device is None or not cuda or t.device == torch.device(device)))
+    if not ok:
+        raise W4A4Error(ERR_INVALID_ARG,
+                        f"{what}: needs a 2-D bfloat16 {'CUDA' if cuda else 'host'} tensor with "
+                        f"unit column stride{' on ' + str(device) if device is not None and cuda else ''}"
+                        f" (got {t.dtype}, shape {tuple(t.shape)}, strides {tuple(t.stride())}, "
+                        f"{t.device})")
+    if not cuda and not t.is_contiguous():
+        raise W4A4Error(ERR_INVALID_ARG, f"{what}: host rows must be dense")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         if not torch.cuda.is_available():
@@ -161,6 +178,7 @@ def workspace_size(T: int, d_in: int, d_out: int, k: int) -> int:
 
 
 def calib_observe(A: torch.Tensor, absmax: torch.Tensor, reset: bool, stream=None):
+    _rows_bf16(A, "calib_observe", absmax.device)
     rows, cols = A.shape
     _check(_calib_observe(_ptr(A), rows, cols, A.stride(0), _ptr(absmax), int(reset),
                           _stream(stream)), "calib_observe")
@@ -219,6 +237,7 @@ def alloc_packed(d_in: int, d_out: int, k: int, layout: int = SF_32x1_KMAJOR, de
 
 
 def pack_weight(W: torch.Tensor, pw: PackedWeight, stream=None):
+    _rows_bf16(W, "pack_weight", pw.wq.device)
     c = pw.c
     _check(_pack_weight(_ptr(W), W.stride(0), _ptr(pw.s), ctypes.byref(c), _stream(stream)),
            "pack_weight")
@@ -261,18 +280,22 @@ def _nz(t: torch.Tensor):
 
 
 def prep_act(X: torch.Tensor, pw: PackedWeight, out: ActBuffers, stream=None):
+    _rows_bf16(X, "prep_act", pw.wq.device)
     c = pw.c
     _check(_prep_act(_ptr(X), X.shape[0], X.stride(0), ctypes.byref(c), _nz(out.aq), _nz(out.sfa),
                      _nz(out.xo), _stream(stream)), "prep_act")
 
 
 def gemm_dual(act: ActBuffers, T: int, pw: PackedWeight, Y: torch.Tensor, stream=None):
+    _rows_bf16(Y, "gemm_dual", pw.wq.device)
     c = pw.c
     _check(_gemm_dual(_nz(act.aq), _nz(act.sfa), _nz(act.xo), T, ctypes.byref(c), _ptr(Y),
                       Y.stride(0), _stream(stream)), "gemm_dual")
 
 
 def linear(X: torch.Tensor, pw: PackedWeight, workspace: torch.Tensor, Y: torch.Tensor, stream=None):
+    _rows_bf16(X, "linear", pw.wq.device)
+    _rows_bf16(Y, "linear", pw.wq.device)
     c = pw.c
     _check(_linear(_ptr(X), X.shape[0], X.stride(0), ctypes.byref(c), _ptr(workspace),
                    workspace.numel() * workspace.element_size(), _ptr(Y), Y.stride(0),
@@ -281,6 +304,12 @@ def linear(X: torch.Tensor, pw: PackedWeight, workspace: torch.Tensor, Y: torch.
 
 def linear_host(X_host: torch.Tensor, pw: PackedWeight, X_dev: torch.Tensor, workspace: torch.Tensor,
                 Y_dev: torch.Tensor, Y_host: torch.Tensor, stream=None):
+    _rows_bf16(X_host, "linear_host", cuda=False)
+    _rows_bf16(Y_host, "linear_host", cuda=False)
+    for t in (X_dev, Y_dev):
+        _rows_bf16(t, "linear_host", pw.wq.device)
+        if not t.is_contiguous():
+            raise W4A4Error(ERR_INVALID_ARG, "linear_host: device rows must be dense")
     c = pw.c
     _check(_linear_host(_ptr(X_host), X_host.shape[0], ctypes.byref(c), _ptr(X_dev),
                         _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -293,6 +322,8 @@ def linear_noalloc(X: torch.Tensor, pw: PackedWeight, Y: torch.Tensor, stream=No
     memory.  Problems larger than NOALLOC_SCRATCH_BYTES of workspace raise
     W4A4Error(ERR_SCRATCH_LIMIT); calls overlapping on the GPU must be
     serialised by the caller (they share the array)."""
+    _rows_bf16(X, "linear_noalloc", pw.wq.device)
+    _rows_bf16(Y, "linear_noalloc", pw.wq.device)
     c = pw.c
     _check(_linear_noalloc(_ptr(X), X.shape[0], X.stride(0), ctypes.byref(c), _ptr(Y), Y.stride(0),
                            _stream(stream)), "linear_noalloc")

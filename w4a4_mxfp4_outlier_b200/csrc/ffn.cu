@@ -162,14 +162,6 @@ extern "C" w4a4_status w4a4_gemm_dual_act(const uint8_t* aq, const uint8_t* sfa,
       (aq_next && !aligned16(aq_next)) || (xo_next && !aligned16(xo_next)))
     return W4A4_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // X_O padding columns k .. k_pad that no output column reaches start at zero
-  if (gn.k_pad > gn.k) {
-    const cudaError_t e = cudaMemset2DAsync(static_cast<uint8_t*>(xo_next) + gn.k * 2,
-                                            static_cast<size_t>(gn.k_pad) * 2, 0,
-                                            static_cast<size_t>(gn.k_pad - gn.k) * 2,
-                                            static_cast<size_t>(T), s);
-    if (e != cudaSuccess) return W4A4_ERR_CUDA;
-  }
   ActOut act;
   act.inv_s = inv_s_perm;
   act.aq = aq_next;
@@ -178,8 +170,20 @@ extern "C" w4a4_status w4a4_gemm_dual_act(const uint8_t* aq, const uint8_t* sfa,
   act.kj = gn.kj;
   act.nblk = gn.nblk;
   act.k_pad = gn.k_pad;
-  return from_cuda(launch_gemm(aq, sfa, xo, T, g, pw->wq, pw->sfb, pw->w_hp, nullptr, g.d_out, s,
-                               &act));
+  // the GEMM's tensor maps are built before anything is enqueued
+  GemmPlan plan;
+  if (plan_gemm(aq, sfa, xo, T, g, pw->wq, pw->sfb, pw->w_hp, nullptr, g.d_out, &act, &plan) !=
+      cudaSuccess)
+    return W4A4_ERR_CUDA;
+  // X_O padding columns k .. k_pad that no output column reaches start at zero
+  if (gn.k_pad > gn.k) {
+    const cudaError_t e = cudaMemset2DAsync(static_cast<uint8_t*>(xo_next) + gn.k * 2,
+                                            static_cast<size_t>(gn.k_pad) * 2, 0,
+                                            static_cast<size_t>(gn.k_pad - gn.k) * 2,
+                                            static_cast<size_t>(T), s);
+    if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  }
+  return from_cuda(run_gemm(plan, s));
 }
 
 extern "C" w4a4_status w4a4_permute_packed_rows(const w4a4_packed_weight* src, const int32_t* rows,

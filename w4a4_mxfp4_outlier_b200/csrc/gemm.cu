@@ -75,29 +75,6 @@ struct GemmSmem {
   uint32_t abort_flag;
 };
 
-struct GemmArgs {
-  const uint8_t* sfa;
-  const uint8_t* sfb;
-  __nv_bfloat16* Y;
-  int64_t ldy;
-  int T;
-  int d_out;
-  int nblk;          // scale blocks per row (kj_pad / 32)
-  int kt_o;          // bf16 K tiles (64 columns each)
-  int kt_j;          // MXFP4 K tiles (256 columns each)
-  int k_pad;         // bf16 columns (multiple of 16)
-  int tiles_m, tiles_n;
-  // Fused FFN epilogue (kernels instantiated with kAct): Y is not stored;
-  // column c of the tile row feeds the next layer, whose input channel c is
-  // its compacted J position c for c < act_kj and outlier c - act_kj after:
-  //   v = fl32(bf16(gelu(bf16(acc))) * act_inv_s[c])
-  // J blocks are MXFP4-encoded into act_aq / act_sfa, outliers go to act_xo.
-  const float* act_inv_s;   // [d_out] inv_s of the next layer in this column order
-  uint8_t* act_aq;          // [T, act_nblk * 16]
-  uint8_t* act_sfa;         // MMA layout, act_nblk blocks per row
-  __nv_bfloat16* act_xo;    // [T, act_k_pad]
-  int act_kj, act_nblk, act_k_pad;
-};
 
 // Accumulator columns as bf16 pairs: the first step of the fused epilogue
 // (bf16(acc), as the plain epilogue would store it), done right after the
@@ -1079,44 +1056,44 @@ static int pair_tile_n(int64_t d_out, bool act) {
 // would be mostly padding).
 constexpr int64_t kPairMinT = 129;
 
-cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
-                        const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
-                        void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act) {
-  if (T == 0 || g.d_out == 0) return cudaSuccess;
-  const bool pair = T >= kPairMinT && pair_capacity() > 0;
-  const int tile_n = pair ? pair_tile_n(g.d_out, act != nullptr) : BN;
+// Host half of a GEMM launch: tile choice, tensor maps and kernel arguments.
+// Enqueues nothing, so a composite call can run it before its first launch and
+// return an error with nothing enqueued.
+cudaError_t plan_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                      const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
+                      void* Y, int64_t ldy, const ActOut* act, GemmPlan* p) {
+  memset(p, 0, sizeof(*p));
+  p->empty = (T == 0 || g.d_out == 0);
+  if (p->empty) return cudaSuccess;
+  p->act = act != nullptr;
+  p->pair = T >= kPairMinT && pair_capacity() > 0;
+  p->tile_n = p->pair ? pair_tile_n(g.d_out, p->act) : BN;
   // B box rows: 256 (single CTA), 128 (pair, 256-wide tile), 64 (pair, 384-wide: 3 boxes)
-  const uint32_t brows = !pair ? BN : (tile_n == 384 ? 64 : 128);
-  CUtensorMap tm_a, tm_b, tm_ao, tm_bo, tm_sfa, tm_sfb;
-  memset(&tm_a, 0, sizeof(tm_a));
-  memset(&tm_b, 0, sizeof(tm_b));
-  memset(&tm_ao, 0, sizeof(tm_ao));
-  memset(&tm_bo, 0, sizeof(tm_bo));
-  memset(&tm_sfa, 0, sizeof(tm_sfa));
-  memset(&tm_sfb, 0, sizeof(tm_sfb));
+  const uint32_t brows = !p->pair ? BN : (p->tile_n == 384 ? 64 : 128);
   const uint64_t row_j = static_cast<uint64_t>(g.kj_pad / 2);
   if (g.kj_pad > 0) {
-    if (!make_tmap(&tm_a, aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, T, row_j, BM) ||
-        !make_tmap(&tm_b, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, g.d_out, row_j, brows))
+    if (!make_tmap(&p->tm_a, aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, T, row_j, BM) ||
+        !make_tmap(&p->tm_b, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_j, g.d_out, row_j, brows))
       return cudaErrorInvalidValue;
-    if (pair) {
+    if (p->pair) {
       // scale buffers seen as rows of 256 bytes; one copy = 4 rows = two 512-byte atoms
       const uint64_t sfa_rows = static_cast<uint64_t>(round_up(T, kSfaRowPad) * g.nblk / 256);
       const uint64_t sfb_rows = static_cast<uint64_t>(g.sfb_rows * g.nblk / 256);
-      if (!make_tmap(&tm_sfa, sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfa_rows, 256, 4, 256,
+      if (!make_tmap(&p->tm_sfa, sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfa_rows, 256, 4, 256,
                      false) ||
-          !make_tmap(&tm_sfb, sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfb_rows, 256, 4, 256,
+          !make_tmap(&p->tm_sfb, sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, sfb_rows, 256, 4, 256,
                      false))
         return cudaErrorInvalidValue;
     }
   }
   if (g.k_pad > 0) {
     const uint64_t row_o = static_cast<uint64_t>(g.k_pad) * 2;
-    if (!make_tmap(&tm_ao, xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, T, row_o, BM) ||
-        !make_tmap(&tm_bo, w_hp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, g.d_out, row_o, brows))
+    if (!make_tmap(&p->tm_ao, xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, T, row_o, BM) ||
+        !make_tmap(&p->tm_bo, w_hp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.k_pad, g.d_out, row_o,
+                   brows))
       return cudaErrorInvalidValue;
   }
-  GemmArgs a;
+  GemmArgs& a = p->a;
   a.sfa = sfa;
   a.sfb = sfb;
   a.Y = static_cast<__nv_bfloat16*>(Y);
@@ -1127,8 +1104,8 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   a.kt_o = static_cast<int>((g.k_pad + 63) / 64);
   a.kt_j = static_cast<int>(g.kj_pad / 256);
   a.k_pad = static_cast<int>(g.k_pad);
-  a.tiles_m = static_cast<int>((T + (pair ? 255 : BM - 1)) / (pair ? 256 : BM));
-  a.tiles_n = static_cast<int>((g.d_out + tile_n - 1) / tile_n);
+  a.tiles_m = static_cast<int>((T + (p->pair ? 255 : BM - 1)) / (p->pair ? 256 : BM));
+  a.tiles_n = static_cast<int>((g.d_out + p->tile_n - 1) / p->tile_n);
   a.act_inv_s = act ? act->inv_s : nullptr;
   a.act_aq = act ? act->aq : nullptr;
   a.act_sfa = act ? act->sfa : nullptr;
@@ -1137,15 +1114,47 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
   a.act_nblk = act ? static_cast<int>(act->nblk) : 0;
   a.act_k_pad = act ? static_cast<int>(act->k_pad) : 0;
   const int ntiles = a.tiles_m * a.tiles_n;
-  if (pair) {
+  if (p->pair) {
     const int npairs = ntiles < pair_capacity() ? ntiles : pair_capacity();
-    const size_t smem = act ? gemm_pair_smem_bytes<true, 256>()
-                            : (tile_n == 384 ? gemm_pair_smem_bytes<false, 384>()
-                                             : gemm_pair_smem_bytes<false, 256>());
+    p->grid = 2 * npairs;
+    p->smem = act ? gemm_pair_smem_bytes<true, 256>()
+                  : (p->tile_n == 384 ? gemm_pair_smem_bytes<false, 384>()
+                                      : gemm_pair_smem_bytes<false, 256>());
+    if (act != nullptr) {
+      // the next layer's codes as tiles of 32 rows x 64 bytes, 64-byte swizzle
+      if (act->nblk > 0 &&
+          !make_tmap(&p->tm_y, act->aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                     static_cast<uint64_t>(act->nblk) * 16, T, static_cast<uint64_t>(act->nblk) * 16,
+                     32, 64, false, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    } else if (!make_tmap(&p->tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
+                          static_cast<uint64_t>(ldy) * 2, 16, 32, false,
+                          CU_TENSOR_MAP_SWIZZLE_64B)) {
+      // Y as bf16 tiles of 16 rows x 32 columns, 64-byte swizzle (epilogue staging layout)
+      return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+  }
+  const int sms = device_num_sms();
+  p->grid = ntiles < sms ? ntiles : sms;
+  p->smem = gemm_smem_bytes();
+  cudaError_t e = p->act ? cudaFuncSetAttribute(gemm_dual_kernel<true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(p->smem))
+                         : cudaFuncSetAttribute(gemm_dual_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(p->smem));
+  return e;
+}
+
+// Device half: enqueues the planned kernel on `stream`.
+cudaError_t run_gemm(const GemmPlan& p, cudaStream_t stream) {
+  if (p.empty) return cudaSuccess;
+  if (p.pair) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * npairs, 1, 1);
+    cfg.gridDim = dim3(p.grid, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = p.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1154,45 +1163,31 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // Y as bf16 tiles of 16 rows x 32 columns, 64-byte swizzle (epilogue staging layout)
-    CUtensorMap tm_y;
-    memset(&tm_y, 0, sizeof(tm_y));
-    if (act != nullptr) {
-      // the next layer's codes as tiles of 32 rows x 64 bytes, 64-byte swizzle
-      if (act->nblk > 0 &&
-          !make_tmap(&tm_y, act->aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
-                     static_cast<uint64_t>(act->nblk) * 16, T, static_cast<uint64_t>(act->nblk) * 16,
-                     32, 64, false, CU_TENSOR_MAP_SWIZZLE_64B))
-        return cudaErrorInvalidValue;
-      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true, 256>, tm_a, tm_b, tm_ao, tm_bo,
-                                tm_sfa, tm_sfb, tm_y, a);
-    }
-    if (!make_tmap(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d_out, T,
-                   static_cast<uint64_t>(ldy) * 2, 16, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
-      return cudaErrorInvalidValue;
-    if (tile_n == 384)
-      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 384>, tm_a, tm_b, tm_ao, tm_bo,
-                                tm_sfa, tm_sfb, tm_y, a);
-    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 256>, tm_a, tm_b, tm_ao, tm_bo,
-                              tm_sfa, tm_sfb, tm_y, a);
+    if (p.act)
+      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true, 256>, p.tm_a, p.tm_b, p.tm_ao,
+                                p.tm_bo, p.tm_sfa, p.tm_sfb, p.tm_y, p.a);
+    if (p.tile_n == 384)
+      return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 384>, p.tm_a, p.tm_b, p.tm_ao,
+                                p.tm_bo, p.tm_sfa, p.tm_sfb, p.tm_y, p.a);
+    return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<false, 256>, p.tm_a, p.tm_b, p.tm_ao,
+                              p.tm_bo, p.tm_sfa, p.tm_sfb, p.tm_y, p.a);
   }
-  const int sms = device_num_sms();
-  const int grid = ntiles < sms ? ntiles : sms;
-  const size_t smem = gemm_smem_bytes();
-  if (act != nullptr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_dual_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    gemm_dual_kernel<true><<<grid, GEMM_THREADS, smem, stream>>>(tm_a, tm_b, tm_ao, tm_bo, a);
-    return cudaGetLastError();
-  }
-  cudaError_t e = cudaFuncSetAttribute(gemm_dual_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  gemm_dual_kernel<false><<<grid, GEMM_THREADS, smem, stream>>>(tm_a, tm_b, tm_ao, tm_bo, a);
+  if (p.act)
+    gemm_dual_kernel<true><<<p.grid, GEMM_THREADS, p.smem, stream>>>(p.tm_a, p.tm_b, p.tm_ao,
+                                                                      p.tm_bo, p.a);
+  else
+    gemm_dual_kernel<false><<<p.grid, GEMM_THREADS, p.smem, stream>>>(p.tm_a, p.tm_b, p.tm_ao,
+                                                                       p.tm_bo, p.a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                        const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
+                        void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act) {
+  GemmPlan p;
+  const cudaError_t e = plan_gemm(aq, sfa, xo, T, g, wq, sfb, w_hp, Y, ldy, act, &p);
+  if (e != cudaSuccess) return e;
+  return run_gemm(p, stream);
 }
 
 }  // namespace w4a4

@@ -61,6 +61,70 @@ static WorkspaceLayout workspace_layout(int64_t T, const Geometry& g) {
   return w;
 }
 
+// Arguments of the activation prep, checked without touching the device.
+static w4a4_status validate_prep(const void* X, int64_t T, int64_t ldx, const Geometry& g,
+                                 const void* aq, const void* sfa, const void* xo) {
+  if (T < 0 || ldx < g.d_in) return W4A4_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 31) - 256) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return W4A4_OK;
+  if (X == nullptr || (g.kj > 0 && (aq == nullptr || sfa == nullptr)) || (g.k > 0 && xo == nullptr))
+    return W4A4_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned16(X) || (aq && !aligned16(aq)) || (sfa && !aligned16(sfa)) ||
+      (xo && !aligned16(xo)))
+    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  return W4A4_OK;
+}
+
+// Arguments of the dual-branch GEMM, checked without touching the device.
+static w4a4_status validate_gemm(const void* aq, const void* sfa, const void* xo, int64_t T,
+                                 const Geometry& g, const void* Y, int64_t ldy) {
+  if (T < 0 || ldy < g.d_out) return W4A4_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 31) - 256) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return W4A4_OK;
+  if (Y == nullptr || (g.kj > 0 && (aq == nullptr || sfa == nullptr)) || (g.k > 0 && xo == nullptr))
+    return W4A4_ERR_INVALID_ARG;
+  if (ldy % 8 != 0 || !aligned16(Y) || (aq && !aligned16(aq)) || (sfa && !aligned16(sfa)) ||
+      (xo && !aligned16(xo)))
+    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  return W4A4_OK;
+}
+
+// The online layer (prep into the workspace at `base`, then the GEMM) as two
+// phases: plan_linear checks every argument of both kernels and builds the
+// GEMM's tensor maps, enqueuing nothing; enqueue_linear launches.  Composite
+// calls run the first before their first enqueue, so a non-OK status always
+// means that nothing was enqueued.
+struct LinearPlan {
+  uint8_t* aq;
+  uint8_t* sfa;
+  void* xo;
+  GemmPlan gemm;
+};
+
+static w4a4_status plan_linear(const void* X, int64_t T, int64_t ldx, const Geometry& g,
+                               const w4a4_packed_weight* pw, uint8_t* base, void* Y, int64_t ldy,
+                               LinearPlan* lp) {
+  const WorkspaceLayout w = workspace_layout(T, g);
+  lp->aq = g.kj > 0 ? base + w.aq : nullptr;
+  lp->sfa = g.kj > 0 ? base + w.sfa : nullptr;
+  lp->xo = g.k > 0 ? base + w.xo : nullptr;
+  w4a4_status st = validate_prep(X, T, ldx, g, lp->aq, lp->sfa, lp->xo);
+  if (st != W4A4_OK) return st;
+  st = validate_gemm(lp->aq, lp->sfa, lp->xo, T, g, Y, ldy);
+  if (st != W4A4_OK) return st;
+  return from_cuda(plan_gemm(lp->aq, lp->sfa, lp->xo, T, g, pw->wq, pw->sfb, pw->w_hp, Y, ldy,
+                             nullptr, &lp->gemm));
+}
+
+static w4a4_status enqueue_linear(const LinearPlan& lp, const void* X, int64_t T, int64_t ldx,
+                                  const Geometry& g, const w4a4_packed_weight* pw,
+                                  cudaStream_t stream) {
+  cudaError_t e = launch_prep(X, T, ldx, pw->inv_s, pw->O, pw->jmap, g, lp.aq, lp.sfa, lp.xo,
+                              stream);
+  if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  return from_cuda(run_gemm(lp.gemm, stream));
+}
+
 }  // namespace w4a4
 
 using namespace w4a4;
@@ -156,14 +220,8 @@ w4a4_status w4a4_prep_act(const void* X, int64_t T, int64_t ldx, const w4a4_pack
   Geometry g;
   w4a4_status st = check_pw(pw, &g);
   if (st != W4A4_OK) return st;
-  if (T < 0 || ldx < g.d_in) return W4A4_ERR_INVALID_ARG;
-  if (T > (int64_t(1) << 31) - 256) return W4A4_ERR_UNSUPPORTED_SHAPE;
-  if (T == 0) return W4A4_OK;
-  if (X == nullptr || (g.kj > 0 && (aq == nullptr || sfa == nullptr)) || (g.k > 0 && xo == nullptr))
-    return W4A4_ERR_INVALID_ARG;
-  if (ldx % 8 != 0 || !aligned16(X) || (aq && !aligned16(aq)) || (sfa && !aligned16(sfa)) ||
-      (xo && !aligned16(xo)))
-    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  st = validate_prep(X, T, ldx, g, aq, sfa, xo);
+  if (st != W4A4_OK || T == 0) return st;
   return from_cuda(launch_prep(X, T, ldx, pw->inv_s, pw->O, pw->jmap, g, aq, sfa, xo,
                                static_cast<cudaStream_t>(stream)));
 }
@@ -173,14 +231,8 @@ w4a4_status w4a4_gemm_dual(const uint8_t* aq, const uint8_t* sfa, const void* xo
   Geometry g;
   w4a4_status st = check_pw(pw, &g);
   if (st != W4A4_OK) return st;
-  if (T < 0 || ldy < g.d_out) return W4A4_ERR_INVALID_ARG;
-  if (T > (int64_t(1) << 31) - 256) return W4A4_ERR_UNSUPPORTED_SHAPE;
-  if (T == 0) return W4A4_OK;
-  if (Y == nullptr || (g.kj > 0 && (aq == nullptr || sfa == nullptr)) || (g.k > 0 && xo == nullptr))
-    return W4A4_ERR_INVALID_ARG;
-  if (ldy % 8 != 0 || !aligned16(Y) || (aq && !aligned16(aq)) || (sfa && !aligned16(sfa)) ||
-      (xo && !aligned16(xo)))
-    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  st = validate_gemm(aq, sfa, xo, T, g, Y, ldy);
+  if (st != W4A4_OK || T == 0) return st;
   return from_cuda(launch_gemm(aq, sfa, xo, T, g, pw->wq, pw->sfb, pw->w_hp, Y, ldy,
                                static_cast<cudaStream_t>(stream)));
 }
@@ -192,17 +244,14 @@ w4a4_status w4a4_linear(const void* X, int64_t T, int64_t ldx, const w4a4_packed
   if (st != W4A4_OK) return st;
   if (T < 0 || ldx < g.d_in || ldy < g.d_out) return W4A4_ERR_INVALID_ARG;
   if (T == 0) return W4A4_OK;
-  const WorkspaceLayout w = workspace_layout(T, g);
-  if (workspace == nullptr || ws_bytes < w.total || X == nullptr || Y == nullptr)
+  if (workspace == nullptr || ws_bytes < workspace_layout(T, g).total || X == nullptr ||
+      Y == nullptr)
     return W4A4_ERR_INVALID_ARG;
   if (!aligned16(workspace)) return W4A4_ERR_UNSUPPORTED_SHAPE;
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint8_t* aq = g.kj > 0 ? base + w.aq : nullptr;
-  uint8_t* sfa = g.kj > 0 ? base + w.sfa : nullptr;
-  void* xo = g.k > 0 ? base + w.xo : nullptr;
-  st = w4a4_prep_act(X, T, ldx, pw, aq, sfa, xo, stream);
+  LinearPlan lp;
+  st = plan_linear(X, T, ldx, g, pw, static_cast<uint8_t*>(workspace), Y, ldy, &lp);
   if (st != W4A4_OK) return st;
-  return w4a4_gemm_dual(aq, sfa, xo, T, pw, Y, ldy, stream);
+  return enqueue_linear(lp, X, T, ldx, g, pw, static_cast<cudaStream_t>(stream));
 }
 
 w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_weight* pw,
@@ -215,14 +264,19 @@ w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_we
   if (T == 0) return W4A4_OK;
   if (X_host == nullptr || Y_host == nullptr || X_dev == nullptr || Y_dev == nullptr)
     return W4A4_ERR_INVALID_ARG;
-  const WorkspaceLayout w = workspace_layout(T, g);
-  if (workspace == nullptr || ws_bytes < w.total) return W4A4_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < workspace_layout(T, g).total) return W4A4_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  // everything the two kernels need is checked (and the GEMM planned) before
+  // the upload is enqueued
+  LinearPlan lp;
+  st = plan_linear(X_dev, T, g.d_in, g, pw, static_cast<uint8_t*>(workspace), Y_dev, g.d_out, &lp);
+  if (st != W4A4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t xb = static_cast<size_t>(T) * static_cast<size_t>(g.d_in) * 2;
   const size_t yb = static_cast<size_t>(T) * static_cast<size_t>(g.d_out) * 2;
   cudaError_t e = cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return W4A4_ERR_CUDA;
-  st = w4a4_linear(X_dev, T, g.d_in, pw, workspace, ws_bytes, Y_dev, g.d_out, stream);
+  st = enqueue_linear(lp, X_dev, T, g.d_in, g, pw, s);
   if (st != W4A4_OK) return st;
   e = cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s);
   return from_cuda(e);

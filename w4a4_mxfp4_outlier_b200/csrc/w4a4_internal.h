@@ -3,6 +3,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "w4a4_device.cuh"
@@ -76,8 +78,46 @@ struct ActOut {
   void* xo;
   int64_t kj, nblk, k_pad;
 };
+// Kernel arguments of the dual-branch GEMM (both kernels of gemm.cu).
+struct GemmArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  __nv_bfloat16* Y;
+  int64_t ldy;
+  int T;
+  int d_out;
+  int nblk;          // scale blocks per row (kj_pad / 32)
+  int kt_o;          // bf16 K tiles (64 columns each)
+  int kt_j;          // MXFP4 K tiles (256 columns each)
+  int k_pad;         // bf16 columns (multiple of 16)
+  int tiles_m, tiles_n;
+  // Fused FFN epilogue (kernels instantiated with kAct): Y is not stored;
+  // column c of the tile row feeds the next layer, whose input channel c is
+  // its compacted J position c for c < act_kj and outlier c - act_kj after:
+  //   v = fl32(bf16(gelu(bf16(acc))) * act_inv_s[c])
+  // J blocks are MXFP4-encoded into act_aq / act_sfa, outliers go to act_xo.
+  const float* act_inv_s;   // [d_out] inv_s of the next layer in this column order
+  uint8_t* act_aq;          // [T, act_nblk * 16]
+  uint8_t* act_sfa;         // MMA layout, act_nblk blocks per row
+  __nv_bfloat16* act_xo;    // [T, act_k_pad]
+  int act_kj, act_nblk, act_k_pad;
+};
+
+// A GEMM launch split in two: plan_gemm does the host work (tile choice,
+// tensor maps, arguments) and enqueues nothing; run_gemm enqueues the kernel.
+struct GemmPlan {
+  CUtensorMap tm_a, tm_b, tm_ao, tm_bo, tm_sfa, tm_sfb, tm_y;
+  GemmArgs a;
+  size_t smem;
+  int grid, tile_n;
+  bool pair, act, empty;
+};
+cudaError_t plan_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
+                      const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
+                      void* Y, int64_t ldy, const ActOut* act, GemmPlan* p);
+cudaError_t run_gemm(const GemmPlan& p, cudaStream_t stream);
 // act == nullptr: Y = bf16 product.  Otherwise Y is not written and the
-// product feeds `act` (see GemmArgs in gemm.cu).
+// product feeds `act` (see GemmArgs).
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,
                         const Geometry& g, const uint8_t* wq, const uint8_t* sfb, const void* w_hp,
                         void* Y, int64_t ldy, cudaStream_t stream, const ActOut* act = nullptr);

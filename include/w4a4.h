@@ -53,7 +53,8 @@ typedef enum w4a4_status {
   W4A4_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
   W4A4_ERR_TIMEOUT = 4,          /* a device pipeline wait ran out (see w4a4_last_error) */
   W4A4_ERR_SCRATCH_LIMIT = 5,    /* the problem needs more scratch than w4a4_linear_noalloc has */
-  W4A4_ERR_BAD_IMAGE = 6         /* a packed-weight image failed its magic, version, size or checksum check */
+  W4A4_ERR_BAD_IMAGE = 6,        /* a packed-weight image failed its magic, version, size or checksum check */
+  W4A4_ERR_NONFINITE_CALIB = 7   /* a calibration magnitude was inf or NaN (see w4a4_calib_finalize) */
 } w4a4_status;
 
 /* Weight scale layouts of the block packing (review sec. 3.4: "32x32 tiles"
@@ -117,7 +118,12 @@ w4a4_status w4a4_calib_observe(const void* A, int64_t rows, int64_t cols, int64_
  *              ascending (int32 [k]);  jmap = the other d_in - k columns
  *              ascending (int32 [d_in - k]).
  * Requires 0 < alpha < 1, 0 <= k <= d_in, 1 <= d_in <= 65535.  O may be NULL
- * when k == 0 and jmap may be NULL when k == d_in. */
+ * when k == 0 and jmap may be NULL when k == d_in.
+ * s is defined for finite magnitudes only: if act_scale or w_scale holds an
+ * inf or a NaN (calibration data that were not finite), the kernel records it
+ * in the device error word -- w4a4_last_error then returns
+ * W4A4_ERR_NONFINITE_CALIB -- and s, inv_s, score, O and jmap are
+ * unspecified. */
 w4a4_status w4a4_calib_finalize(const float* act_scale, const float* w_scale, int64_t d_in,
                                 double alpha, int64_t k, float* s, float* inv_s, float* score,
                                 int32_t* O, int32_t* jmap, void* stream);
@@ -176,6 +182,13 @@ w4a4_status w4a4_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int64_t 
  * Each 32-element block takes e = clamp(floor(log2 amax) - 2, -127, 127),
  * code = e + 127 (0 for an all-zero block), elements v * 2^-e rounded to
  * E2M1 (nearest, ties to even, saturating at 6, sign kept).
+ * Non-finite values (inf or NaN in X, or a product x * inv_s beyond the
+ * float32 range, which is +-inf) follow IEEE float32 arithmetic: amax is the
+ * NaN-propagating maximum of |v|; a block holding a NaN gets scale code 0xFF
+ * (E8M0's NaN) and all-zero element codes; a block holding an infinity (and
+ * no NaN) gets e = 127 (code 254), its infinities saturate to +-6 and its
+ * finite elements are v * 2^-127 on the E2M1 grid; an outlier column takes
+ * bf16_rn(v): +-inf stays +-inf and every NaN is written as 0x7FC0.
  * aq, sfa, xo may be NULL when their size is zero. */
 w4a4_status w4a4_prep_act(const void* X, int64_t T, int64_t ldx, const w4a4_packed_weight* pw,
                           uint8_t* aq, uint8_t* sfa, void* xo, void* stream);
@@ -346,8 +359,9 @@ w4a4_status w4a4_error_sums(const void* Y, int64_t ldy, const float* Yref, int64
                             int64_t d_out, double* sums, void* stream);
 
 /* Synchronises `stream` and reports device-side failures recorded since the
- * last clear: W4A4_OK, or W4A4_ERR_TIMEOUT if a bounded wait ran out (the
- * affected output is incomplete).  *bits (may be NULL) receives the raw
+ * last clear: W4A4_OK, W4A4_ERR_TIMEOUT if a bounded wait ran out (the
+ * affected output is incomplete; reported first), or W4A4_ERR_NONFINITE_CALIB
+ * if w4a4_calib_finalize met an inf or NaN magnitude.  *bits (may be NULL) receives the raw
  * error word.  clear != 0 resets the word. */
 w4a4_status w4a4_last_error(void* stream, int clear, uint32_t* bits);
 

@@ -40,7 +40,18 @@ notes):
 * an all-zero block gets scale code 0 (2^-127) and +-0 codes; the sign of
   zero is kept (code 0x8 for -0);
 * the high-precision branch is bfloat16 with round-to-nearest-even;
-* nibble order: element 2i in bits [3:0] of byte i, 2i+1 in bits [7:4].
+* nibble order: element 2i in bits [3:0] of byte i, 2i+1 in bits [7:4];
+* non-finite values follow IEEE float32 arithmetic and the E8M0 encoding:
+  v = fl32(x * inv_s) is +-inf for an infinite x or a product beyond the
+  float32 range and NaN for a NaN x; a block's amax is the NaN-propagating
+  maximum of |v|; amax = NaN gives scale code 0xFF (E8M0's NaN, the one code
+  that marks a whole block as NaN) and all-zero element codes; amax = +inf
+  gives e = clamp(floor(log2 inf) - 2) = 127 (code 254), infinities saturate
+  to +-6 and finite elements take v * 2^-127 on the E2M1 grid; the bf16
+  branch keeps +-inf and writes every NaN as 0x7FC0 (the quiet NaN without
+  payload: IEEE does not fix a NaN's sign or payload);
+* calibration magnitudes must be finite: s_j is undefined for an infinite or
+  NaN magnitude, and the oracle refuses to compute it.
 
 Precision: bf16 inputs are exact in float32.  Every product the method
 defines (x * inv_s, w * s) is one float32 multiply with round-to-nearest
@@ -75,7 +86,8 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float32 -> bfloat16 bit patterns, round to nearest, ties to even."""
+    """float32 -> bfloat16 bit patterns, round to nearest, ties to even;
+    +-inf stay +-inf, every NaN becomes 0x7FC0 (quiet, no payload)."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
     lsb = (u >> 16) & 1
     r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
@@ -205,6 +217,8 @@ def smoothing_factors(act_scale: np.ndarray, w_scale: np.ndarray, alpha: float):
     rounded once to float32.  inv_s = fl32(1 / s) is what the online path
     multiplies by.  Returns (s, inv_s) as float32 arrays.
     """
+    if not (np.all(np.isfinite(act_scale)) and np.all(np.isfinite(w_scale))):
+        raise ValueError("calibration magnitudes must be finite: s_j is undefined for inf or NaN")
     a = np.maximum(act_scale.astype(np.float64), SCALE_FLOOR)
     w = np.maximum(w_scale.astype(np.float64), SCALE_FLOOR)
     s64 = np.power(a, float(alpha)) / np.power(w, 1.0 - float(alpha))
@@ -255,14 +269,17 @@ def select_outliers(score: np.ndarray, k: int):
 # ----------------------------------------------------------------------------
 
 def mx_shared_exponent(amax: np.ndarray) -> np.ndarray:
-    """e = floor(log2 amax) - 2 clamped to [-127, 127]; e = -127 for amax = 0.
+    """e = floor(log2 amax) - 2 clamped to [-127, 127]; e = -127 for amax = 0;
+    e = 127 for amax = +inf (floor(log2 inf) is +inf, which the clamp takes to
+    127).  A NaN amax has no exponent; the caller codes such a block as NaN.
 
     floor(log2 amax) is read exactly from frexp (amax = m 2^ex, m in [0.5,1)).
     """
     amax = np.asarray(amax, dtype=np.float64)
-    _, ex = np.frexp(amax)
+    _, ex = np.frexp(np.where(np.isfinite(amax), amax, 1.0))
     e = ex.astype(np.int64) - 1 - E2M1_EMAX
     e = np.where(amax == 0.0, -E8M0_BIAS, e)
+    e = np.where(np.isposinf(amax), 127, e)
     return np.clip(e, -127, 127)
 
 
@@ -290,10 +307,18 @@ def mxfp4_quantize_blocks(V: np.ndarray, block_amax: np.ndarray | None = None):
     """
     V = np.asarray(V, dtype=np.float32)
     if block_amax is None:
-        block_amax = np.max(np.abs(V), axis=-1)
-    e = mx_shared_exponent(block_amax)
-    q = np.ldexp(V, (-e)[..., None].astype(np.int32)).astype(np.float32)  # exact
-    return (e + E8M0_BIAS).astype(np.uint8), e2m1_codes(q)
+        block_amax = np.max(np.abs(V), axis=-1)           # NaN if the block holds a NaN
+    nan_block = np.isnan(block_amax)
+    e = mx_shared_exponent(np.where(nan_block, 0.0, block_amax))
+    # q = v 2^-e is exact in float32 except below 2^-126 (only for e = 127),
+    # where it rounds to a subnormal: far below 0.25, the smallest rounding
+    # boundary of the E2M1 grid, so the codes are those of the exact q
+    with np.errstate(under="ignore", over="ignore", invalid="ignore"):
+        q = np.ldexp(V, (-e)[..., None].astype(np.int32)).astype(np.float32)
+        codes = e2m1_codes(q)
+    codes = np.where(nan_block[..., None], np.uint8(0), codes).astype(np.uint8)
+    scale = np.where(nan_block, 0xFF, e + E8M0_BIAS).astype(np.uint8)
+    return scale, codes
 
 
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:
@@ -321,6 +346,7 @@ def dequant_mxfp4(packed: np.ndarray, sf: np.ndarray, ncols: int | None = None) 
     codes = unpack_nibbles(packed)
     K = codes.shape[-1]
     scale = np.ldexp(1.0, sf.astype(np.int64) - E8M0_BIAS)          # 2^(sf-127)
+    scale = np.where(sf == 0xFF, np.nan, scale)                      # E8M0 0xFF is NaN
     vals = e2m1_value(codes) * np.repeat(scale, MX_BLOCK, axis=-1)[..., :K]
     return vals if ncols is None else vals[..., :ncols]
 
@@ -359,7 +385,8 @@ def prep_activation(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray, J: np.ndarr
     inv_s = inv_s.astype(np.float32)
     for r0 in range(0, T, row_chunk):
         r1 = min(T, r0 + row_chunk)
-        V = smooth_activation(X[r0:r1].astype(np.float32), inv_s)     # fl32 products
+        with np.errstate(over="ignore", invalid="ignore"):
+            V = smooth_activation(X[r0:r1].astype(np.float32), inv_s)   # fl32 products (may be +-inf)
         xo[r0:r1] = f32_to_bf16_bits(V[:, O])
         if nb:
             VJ = _pad_cols(V[:, J], nb * MX_BLOCK).reshape(r1 - r0, nb, MX_BLOCK)
@@ -396,7 +423,8 @@ def pack_weight(W: np.ndarray, s: np.ndarray, O: np.ndarray, J: np.ndarray,
     w_hp = np.zeros((d_out, O.shape[0]), np.uint16)
     for r0 in range(0, d_out, row_chunk):
         r1 = min(d_out, r0 + row_chunk)
-        Wf = fold_weight(W[r0:r1].astype(np.float32), s).astype(np.float32)   # fl32 products
+        with np.errstate(over="ignore", invalid="ignore"):
+            Wf = fold_weight(W[r0:r1].astype(np.float32), s).astype(np.float32)   # fl32 products
         w_hp[r0:r1] = f32_to_bf16_bits(Wf[:, O])
         if not nb:
             continue

@@ -304,7 +304,53 @@ def _pack_zero_in_place(W, s, O, J, layout=orc.LAYOUT_32x1, row_chunk=512):
     return out
 
 
+def _block_amax_ignores_nan(V, block_amax=None):
+    """Block maximum that skips NaNs (numpy's nanmax) instead of propagating them."""
+    if block_amax is None:
+        with np.errstate(invalid="ignore"):
+            block_amax = np.nanmax(np.abs(np.asarray(V, dtype=np.float32)), axis=-1)
+        block_amax = np.where(np.isnan(block_amax), 0.0, block_amax)
+    return _orig["mxfp4_quantize_blocks"](V, block_amax)
+
+
+def _exponent_inf_126(amax):
+    """An infinite maximum read as the exponent field 255 (e = 255 - 127 - 2)."""
+    e = _orig["mx_shared_exponent"](amax)
+    return np.where(np.isposinf(np.asarray(amax, dtype=np.float64)), 126, e)
+
+
+def _dequant_nan_scale_finite(packed, sf, ncols=None):
+    """E8M0 0xFF read as 2^128 instead of NaN."""
+    codes = orc.unpack_nibbles(packed)
+    K = codes.shape[-1]
+    scale = np.ldexp(1.0, sf.astype(np.int64) - orc.E8M0_BIAS)
+    vals = orc.e2m1_value(codes) * np.repeat(scale, orc.MX_BLOCK, axis=-1)[..., :K]
+    return vals if ncols is None else vals[..., :ncols]
+
+
+def _bf16_nan_keeps_sign(x):
+    """A NaN keeps its sign bit in bf16 (0xFFC0 for -NaN)."""
+    bits = _orig["f32_to_bf16_bits"](x)
+    neg = np.signbit(np.asarray(x, dtype=np.float32)) & np.isnan(np.asarray(x, dtype=np.float32))
+    return np.where(neg, np.uint16(0xFFC0), bits)
+
+
+def _smoothing_accepts_nonfinite(act_scale, w_scale, alpha):
+    """s computed from infinite or NaN magnitudes instead of refused."""
+    a = np.maximum(act_scale.astype(np.float64), orc.SCALE_FLOOR)
+    w = np.maximum(w_scale.astype(np.float64), orc.SCALE_FLOOR)
+    with np.errstate(invalid="ignore", over="ignore", divide="ignore"):
+        s = (np.power(a, float(alpha)) / np.power(w, 1.0 - float(alpha))).astype(np.float32)
+        inv_s = (1.0 / s.astype(np.float64)).astype(np.float32)
+    return s, inv_s
+
+
 MUTANTS = {
+    "block_amax_ignores_nan": {"mxfp4_quantize_blocks": _block_amax_ignores_nan},
+    "exponent_inf_126": {"mx_shared_exponent": _exponent_inf_126},
+    "dequant_nan_scale_finite": {"dequant_mxfp4": _dequant_nan_scale_finite},
+    "bf16_nan_keeps_sign": {"f32_to_bf16_bits": _bf16_nan_keeps_sign},
+    "smoothing_accepts_nonfinite": {"smoothing_factors": _smoothing_accepts_nonfinite},
     "zero_in_place": {"prep_activation": _prep_zero_in_place, "pack_weight": _pack_zero_in_place},
     "gelu_double_round": {"gelu_bf16": _gelu_double_round},
     "no_scale_floor": {"smoothing_factors": _no_scale_floor},

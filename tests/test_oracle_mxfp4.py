@@ -155,3 +155,31 @@ def test_mma_scale_layout_is_a_bijection():
     # the second K atom of row-block 0 starts at byte 512, row-block 1 after all K atoms
     assert orc.mma_sf_offset(0, 4, nblk) == 512
     assert orc.mma_sf_offset(128, 0, nblk) == 1024
+
+
+def test_dequant_of_the_non_finite_scale_codes():
+    # E8M0: code 254 is 2^127, the largest scale; 0xFF is NaN and makes its
+    # whole block NaN, whatever the element codes (here all zero)
+    codes = np.zeros((2, 32), np.uint8)
+    codes[0, :3] = [0x7, 0xF, 0x2]                    # 6, -6, 1
+    sf = np.array([[254], [255]], np.uint8)
+    deq = orc.dequant_mxfp4(orc.pack_nibbles(codes), sf)
+    assert deq[0, 0] == 6.0 * 2.0 ** 127 and deq[0, 1] == -6.0 * 2.0 ** 127
+    assert deq[0, 2] == 2.0 ** 127 and deq[0, 3] == 0.0
+    assert np.isnan(deq[1]).all()
+
+
+def test_nan_and_inf_blocks_among_finite_ones():
+    # a row of three blocks: finite, holding an infinity, holding a NaN --
+    # each block is coded on its own, the finite one exactly as if alone
+    rng = np.random.default_rng(2)
+    V = rng.normal(size=(1, 3, 32)).astype(np.float32)
+    alone_sc, alone_codes = orc.mxfp4_quantize_blocks(V[:, 0])
+    V[0, 1, 7] = -np.inf
+    V[0, 2, 30] = np.nan
+    sc, codes = orc.mxfp4_quantize_blocks(V)
+    assert sc[0, 0] == alone_sc[0] and (codes[0, 0] == alone_codes[0]).all()
+    assert sc[0, 1] == 254 and codes[0, 1, 7] == 0xF
+    # the block's finite normals, scaled by 2^-127, all lie below 0.25
+    assert ((codes[0, 1, np.arange(32) != 7] & 7) == 0).all()
+    assert sc[0, 2] == 255 and not codes[0, 2].any()

@@ -368,3 +368,49 @@ def test_smoothing_and_splitting_help():
     plain = orc.dual_branch_product(pa["aq"], pa["sfa"], pa["xo"], pw["wq"], pw["sfb"], pw["w_hp"])
     ours, _ = orc.linear_reference(X, W, 0.5, 8)
     assert snr(ours) > snr(plain)
+
+
+def test_non_finite_activations_hand_worked():
+    # Where the pages say nothing, IEEE float32 arithmetic and the E8M0 codes
+    # decide (see the oracle's readings).  d_in = 64, O = {0, 1}: X_O holds
+    # columns 0 and 1; J = 2 .. 63 forms block 0 (columns 2 .. 33) and block 1
+    # (34 .. 63 and two zeros).  Values worked by hand:
+    #  row 0: x00 = 2^127 times inv_s 4 overflows -> +inf -> bf16 0x7F80;
+    #         x01 = NaN -> 0x7FC0; x02 = -inf -> block 0 amax inf, e = 127
+    #         (code 254), code 0xF; x03 = 1.5 2^126 -> q = 0.75 -> code 2;
+    #         x04 = 1 -> q = 2^-127 -> code 0; x34 = NaN -> block 1 code 255,
+    #         all codes 0.
+    #  row 1: x05 = 2^127 times inv_s 2 -> 2^128 overflows -> +inf: block 0
+    #         code 254, its code (position 3) 7; x06 = -2^126 -> q = -0.5 ->
+    #         code 9; x01 = -NaN (sign set) -> still 0x7FC0; block 1 all zero
+    #         -> code 0.
+    d_in = 64
+    O = np.array([0, 1], np.int32)
+    J = np.arange(2, d_in, dtype=np.int32)
+    inv_s = np.ones(d_in, np.float32)
+    inv_s[0] = 4.0
+    inv_s[5] = 2.0
+    X = np.zeros((2, d_in), np.float32)
+    X[0, [0, 1, 2, 3, 4, 34]] = [2.0 ** 127, np.nan, -np.inf, 1.5 * 2.0 ** 126, 1.0, np.nan]
+    X[1, [1, 5, 6]] = [-np.nan, 2.0 ** 127, -2.0 ** 126]
+    out = orc.prep_activation(X, inv_s, O, J)
+    assert out["xo"][0].tolist() == [0x7F80, 0x7FC0]
+    assert out["xo"][1].tolist() == [0x0000, 0x7FC0]
+    assert out["sfa"].tolist() == [[254, 255], [254, 0]]
+    codes = orc.unpack_nibbles(out["aq"])
+    assert codes[0, :3].tolist() == [0xF, 0x2, 0x0] and not codes[0, 3:].any()
+    assert codes[1, :5].tolist() == [0, 0, 0, 0x7, 0x9] and not codes[1, 5:].any()
+
+
+def test_calibration_refuses_non_finite_magnitudes():
+    # s_j = a^alpha / w^(1 - alpha) has no value for an infinite or NaN magnitude
+    a = np.ones(8, np.float32)
+    w = np.ones(8, np.float32)
+    for bad in (np.inf, np.nan):
+        for which in ("act", "w"):
+            aa, ww = a.copy(), w.copy()
+            (aa if which == "act" else ww)[3] = bad
+            with pytest.raises(ValueError):
+                orc.smoothing_factors(aa, ww, 0.5)
+    s, inv_s = orc.smoothing_factors(a, w, 0.5)
+    assert (s == 1).all() and (inv_s == 1).all()

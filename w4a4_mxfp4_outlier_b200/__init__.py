@@ -25,7 +25,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 (OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT,
- ERR_BAD_IMAGE) = range(7)
+ ERR_BAD_IMAGE, ERR_NONFINITE_CALIB) = range(8)
 NOALLOC_SCRATCH_BYTES = 32 << 20     # W4A4_NOALLOC_SCRATCH_BYTES
 SF_32x1_KMAJOR, SF_32x32_TILE, SF_128x1_KMAJOR = 0, 1, 2
 

@@ -108,6 +108,10 @@ __global__ void finalize_scales_kernel(const float* __restrict__ act, const floa
                                        float* __restrict__ inv_s, float* __restrict__ score) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d_in) return;
+  // s is defined for finite magnitudes only: an infinite or NaN one (from
+  // non-finite calibration data) is reported, and that column's s, inv_s,
+  // score and the selection are then unspecified
+  if (!isfinite(act[j]) || !isfinite(wsc[j])) atomicOr(&g_device_error, DEVERR_NONFINITE_CALIB);
   const double a = fmax(static_cast<double>(act[j]), 1e-5);
   const double w = fmax(static_cast<double>(wsc[j]), 1e-5);
   const float sj = static_cast<float>(pow(a, alpha) / pow(w, 1.0 - alpha));

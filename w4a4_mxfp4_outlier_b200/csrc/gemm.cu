@@ -151,7 +151,8 @@ __device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0,
     for (int i = 0; i < 32; ++i) {
       const int o = col0 + i - a.act_kj;
       const float vi = (i & 1) ? v[i >> 1].y : v[i >> 1].x;
-      if (o >= 0 && o < a.act_k_pad) xr[o] = __float2bfloat16_rn(vi);
+      if (o >= 0 && o < a.act_k_pad)
+        xr[o] = __ushort_as_bfloat16(static_cast<unsigned short>(bf16_rn_bits(vi)));
     }
   }
   // the MX block of compacted positions col0 .. col0+31 (zeros past act_kj)
@@ -166,9 +167,7 @@ __device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0,
         }
       }
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+    const float amax = block_absmax32(v);   // NaN if any element is NaN
     const uint32_t code = mx_scale_code(amax);
     const float inv = mx_inv_scale(code);
     const float2 inv2 = make_float2(inv, inv);
@@ -177,7 +176,7 @@ __device__ __noinline__ uint32_t act_block(const BfPairs16 y, int row, int col0,
     for (int q = 0; q < 4; ++q) {
       const float2 a0 = __fmul2_rn(v[4 * q], inv2), a1 = __fmul2_rn(v[4 * q + 1], inv2);
       const float2 a2 = __fmul2_rn(v[4 * q + 2], inv2), a3 = __fmul2_rn(v[4 * q + 3], inv2);
-      w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y);
+      w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y) & mx_nan_block_mask(code);
     }
     if (stg != 0u) {
       // the staging row of this lane: 16-byte chunk (b & 3) at the 64-byte

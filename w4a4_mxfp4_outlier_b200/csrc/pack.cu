@@ -42,11 +42,11 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
       x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[src_row * ldw + j]) << 16), s[j]);
     }
     v[i] = x;
-    amax = fmaxf(amax, fabsf(x));
+    amax = max_nan(amax, fabsf(x));       // NaN-propagating
   }
   if (layout == 1) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    for (int o = 16; o > 0; o >>= 1) amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
   }
   const uint32_t code = mx_scale_code(amax);
   const float inv = mx_inv_scale(code);
@@ -56,7 +56,8 @@ __global__ void __launch_bounds__(256) pack_j_kernel(const uint16_t* __restrict_
     for (int q = 0; q < 4; ++q)
       w[q] = cvt_e2m1x8(v[8 * q] * inv, v[8 * q + 1] * inv, v[8 * q + 2] * inv, v[8 * q + 3] * inv,
                         v[8 * q + 4] * inv, v[8 * q + 5] * inv, v[8 * q + 6] * inv,
-                        v[8 * q + 7] * inv);
+                        v[8 * q + 7] * inv) &
+             mx_nan_block_mask(code);
     const int64_t row_bytes = static_cast<int64_t>(nblk) * 16;
     *reinterpret_cast<uint4*>(wq + static_cast<int64_t>(n) * row_bytes + b * 16) =
         make_uint4(w[0], w[1], w[2], w[3]);
@@ -79,7 +80,7 @@ __global__ void pack_o_kernel(const uint16_t* __restrict__ W, int64_t ldw,
     const int64_t src_row = rows ? rows[n] : n;
     x = __fmul_rn(__uint_as_float(static_cast<uint32_t>(W[src_row * ldw + j]) << 16), s[j]);
   }
-  w_hp[idx] = __float2bfloat16_rn(x);
+  w_hp[idx] = __ushort_as_bfloat16(static_cast<unsigned short>(bf16_rn_bits(x)));
 }
 
 cudaError_t launch_pack(const void* W, int64_t ldw, const float* s, const int32_t* O,

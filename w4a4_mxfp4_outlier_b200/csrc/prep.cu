@@ -197,13 +197,13 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
             const float x0 = __uint_as_float(ring_bf16(ring, go[c][2 * q]));
             const float x1 = __uint_as_float(ring_bf16(ring, go[c][2 * q + 1]));
             v[q] = __fmul2_rn(make_float2(x0, x1), isv[c][q]);
-            amax = fmaxf(amax, fmaxf(fabsf(v[q].x), fabsf(v[q].y)));
+            amax = max3_nan(amax, fabsf(v[q].x), fabsf(v[q].y));   // NaN-propagating
           }
-          amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-          amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+          amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+          amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
           if (stripe4) {                      // 128x1 stripes: 16 lanes, 4 blocks
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 8));
+            amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+            amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 8));
           }
           const uint32_t code = mx_scale_code(amax);
           const float inv = mx_inv_scale(code);
@@ -212,7 +212,7 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
 #pragma unroll
           for (int q = 0; q < 4; ++q) qv[q] = __fmul2_rn(v[q], inv2);
           uint32_t w = cvt_e2m1x8(qv[0].x, qv[0].y, qv[1].x, qv[1].y, qv[2].x, qv[2].y, qv[3].x,
-                                  qv[3].y);
+                                  qv[3].y) & mx_nan_block_mask(code);
           w = __funnelshift_l(w, w, 8 * rot);   // undo the pair rotation
           *reinterpret_cast<uint32_t*>(aq_p + 4 * chunk) = w;
           const uint32_t c4 = __shfl_down_sync(0xFFFFFFFFu, code, 4);
@@ -229,8 +229,7 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
         const float x0 = __uint_as_float(ring_bf16(ring, oo0));
         const float x1 = __uint_as_float(ring_bf16(ring, oo1));
         const float2 v = __fmul2_rn(make_float2(x0, x1), oinv);
-        xo_p[ct] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+        xo_p[ct] = bf16_rn_bits(v.x) | (bf16_rn_bits(v.y) << 16);
         for (int i2 = ct + NT; i2 < xo_row; i2 += NT) {
           const int o0 = 2 * i2;
           const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : kPrepZero;
@@ -238,8 +237,7 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
           const float y0 = __fmul_rn(__uint_as_float(ring_bf16(ring, a0)), o0 < k ? inv_s[O[o0]] : 1.f);
           const float y1 =
               __fmul_rn(__uint_as_float(ring_bf16(ring, a1)), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
-          xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
-                     (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+          xo_p[i2] = bf16_rn_bits(y0) | (bf16_rn_bits(y1) << 16);
         }
       }
       __syncwarp();

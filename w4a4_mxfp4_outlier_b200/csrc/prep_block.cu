@@ -192,28 +192,23 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         for (int e = 0; e < 16; ++e)
           v[e] = __fmul2_rn(make_float2(pb_ring_f32(ring, go[2 * e]), pb_ring_f32(ring, go[2 * e + 1])),
                             isv[e]);
-        float mx[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          mx[e] = fmaxf(fmaxf(fabsf(v[2 * e].x), fabsf(v[2 * e].y)),
-                        fmaxf(fabsf(v[2 * e + 1].x), fabsf(v[2 * e + 1].y)));
-        amax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        amax = block_absmax32(v);            // NaN if any element is NaN
       }
       if (stripe4) {                        // 128x1 stripes: the 4 lanes of 4 consecutive blocks
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = max_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
       }
       if (enc) {
         const uint32_t code = mx_scale_code(amax);
         const float inv = mx_inv_scale(code);
         const float2 inv2 = make_float2(inv, inv);
+        const uint32_t keep = mx_nan_block_mask(code);
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 a0 = __fmul2_rn(v[4 * q], inv2), a1 = __fmul2_rn(v[4 * q + 1], inv2);
           const float2 a2 = __fmul2_rn(v[4 * q + 2], inv2), a3 = __fmul2_rn(v[4 * q + 3], inv2);
-          w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y);
+          w[q] = cvt_e2m1x8(a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y) & keep;
         }
         // nibble e holds element (e + rot) mod 32: rotate the 128 bits left by
         // 4 * rot = 32 * ws + bs bits
@@ -244,16 +239,14 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         const float x0 = pb_ring_f32(ring, oo0);
         const float x1 = pb_ring_f32(ring, oo1);
         const float2 vv = __fmul2_rn(make_float2(x0, x1), oinv);
-        xo_p[t] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(vv.x))) |
-                  (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(vv.y))) << 16);
+        xo_p[t] = bf16_rn_bits(vv.x) | (bf16_rn_bits(vv.y) << 16);
         for (int i2 = t + ntg; i2 < xo_row; i2 += ntg) {
           const int o0 = 2 * i2;
           const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : R::kZero;
           const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : R::kZero;
           const float y0 = __fmul_rn(pb_ring_f32(slot, a0), o0 < k ? inv_s[O[o0]] : 1.f);
           const float y1 = __fmul_rn(pb_ring_f32(slot, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
-          xo_p[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y0))) |
-                     (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+          xo_p[i2] = bf16_rn_bits(y0) | (bf16_rn_bits(y1) << 16);
         }
       }
       __syncwarp();

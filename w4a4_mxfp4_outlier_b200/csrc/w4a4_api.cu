@@ -142,6 +142,7 @@ const char* w4a4_status_string(w4a4_status s) {
     case W4A4_ERR_TIMEOUT: return "device pipeline wait timed out";
     case W4A4_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed no-alloc scratch";
     case W4A4_ERR_BAD_IMAGE: return "packed-weight image failed its header or checksum check";
+    case W4A4_ERR_NONFINITE_CALIB: return "a calibration magnitude was inf or NaN";
   }
   return "unknown status";
 }
@@ -294,10 +295,10 @@ w4a4_status w4a4_last_error(void* stream, int clear, uint32_t* bits) {
     if (e != cudaSuccess) return W4A4_ERR_CUDA;
   }
   if (bits) *bits = v;
-  return (v & (DEVERR_TIMEOUT_PRODUCER | DEVERR_TIMEOUT_MMA | DEVERR_TIMEOUT_EPILOGUE |
-               DEVERR_TIMEOUT_PREP))
-             ? W4A4_ERR_TIMEOUT
-             : W4A4_OK;
+  if (v & (DEVERR_TIMEOUT_PRODUCER | DEVERR_TIMEOUT_MMA | DEVERR_TIMEOUT_EPILOGUE |
+           DEVERR_TIMEOUT_PREP))
+    return W4A4_ERR_TIMEOUT;
+  return (v & DEVERR_NONFINITE_CALIB) ? W4A4_ERR_NONFINITE_CALIB : W4A4_OK;
 }
 
 }  // extern "C"

@@ -19,6 +19,7 @@ enum : uint32_t {
   DEVERR_TIMEOUT_MMA = 1u << 1,
   DEVERR_TIMEOUT_EPILOGUE = 1u << 2,
   DEVERR_TIMEOUT_PREP = 1u << 3,
+  DEVERR_NONFINITE_CALIB = 1u << 4,   // calibration magnitude was inf or NaN
   DEVERR_BAD_ARG = 1u << 8,
 };
 // The library is compiled as one translation unit (csrc/libw4a4.cu), so this
@@ -526,18 +527,64 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, flo
   return r;
 }
 
-// E8M0 scale code for a block maximum: clamp(floor(log2 amax) - 2, -127, 127)
-// + 127, read from the exponent field (0 for zero / subnormal maxima).
-__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
-  const int ebits = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
-  int e = ebits - 127 - 2;
-  e = e < -127 ? -127 : e;
-  return static_cast<uint32_t>(e + 127);
+// Maxima of magnitudes with NaN propagation (IEEE 754-2019 maximum): the
+// maximum of a block that holds a NaN is NaN, of one that holds an infinity
+// (and no NaN) +inf.  Three-input form: one instruction for three values.
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
-// 2^-e as a float for the scale code c = e + 127 (e in [-127, 125]).
+// max |v| over 32 values, NaN-propagating (16 instructions)
+__device__ __forceinline__ float block_absmax32(const float2 (&v)[16]) {
+  float m[12];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    m[2 * i] = max3_nan(fabsf(v[3 * i].x), fabsf(v[3 * i].y), fabsf(v[3 * i + 1].x));
+    m[2 * i + 1] = max3_nan(fabsf(v[3 * i + 1].y), fabsf(v[3 * i + 2].x), fabsf(v[3 * i + 2].y));
+  }
+  m[10] = fabsf(v[15].x);
+  m[11] = fabsf(v[15].y);
+  const float n0 = max3_nan(m[0], m[1], m[2]), n1 = max3_nan(m[3], m[4], m[5]);
+  const float n2 = max3_nan(m[6], m[7], m[8]), n3 = max3_nan(m[9], m[10], m[11]);
+  return max_nan(max3_nan(n0, n1, n2), n3);
+}
+
+// E8M0 scale code for a block maximum amax (>= 0, +inf or NaN):
+// clamp(floor(log2 amax) - 2, -127, 127) + 127, read from the exponent field
+// (0 for zero / subnormal maxima).  amax = +inf gives e = 127, code 254;
+// amax = NaN gives 0xFF, E8M0's NaN, and the block's element codes are all
+// zero (mx_nan_block_mask).
+__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
+  const uint32_t b = __float_as_uint(amax) & 0x7FFFFFFFu;
+  const uint32_t ebits = b >> 23;
+  if (ebits == 255u) return b == 0x7F800000u ? 254u : 255u;
+  return ebits > 2u ? ebits - 2u : 0u;
+}
+
+// 2^-e as a float for the scale code c = e + 127: exact for e <= 126, and
+// 2^-127 (a subnormal float) for code 254 (and for the NaN code, whose
+// element codes are zeroed anyway).
 __device__ __forceinline__ float mx_inv_scale(uint32_t code) {
-  return __uint_as_float((254u - code) << 23);
+  return __uint_as_float(code < 254u ? (254u - code) << 23 : 0x00400000u);
+}
+
+// AND mask for a block's code words: 0 for a NaN block (scale code 0xFF).
+__device__ __forceinline__ uint32_t mx_nan_block_mask(uint32_t code) {
+  return code == 255u ? 0u : 0xFFFFFFFFu;
+}
+
+// bf16 bits of v rounded to nearest even; every NaN becomes 0x7FC0, the
+// quiet NaN without payload (a NaN's sign and payload are not carried).
+__device__ __forceinline__ uint32_t bf16_rn_bits(float v) {
+  const uint32_t b = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+  return v != v ? 0x7FC0u : b;
 }
 
 }  // namespace w4a4

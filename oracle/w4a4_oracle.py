@@ -508,7 +508,8 @@ def search_layer(X: np.ndarray, W: np.ndarray, alphas, ks, layouts=(LAYOUT_32x1,
     alpha and k"; sec. 6 "next step"; no procedure given]: for every
     candidate the quantised layer's Y on X_eval (default X, calibration on X)
     is compared with the exact float64 product X_eval W^T; the smallest
-    relative Frobenius error wins, the smaller k on ties.
+    relative Frobenius error wins, the smaller k on ties, then the candidate
+    listed first (layouts, then k, then alpha, in the order given).
     Returns (best, {candidate: error})."""
     Xe = X if X_eval is None else X_eval
     exact = Xe.astype(np.float64) @ W.astype(np.float64).T

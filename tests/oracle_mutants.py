@@ -19,7 +19,7 @@ _orig = {name: getattr(orc, name) for name in (
     "smoothing_factors", "outlier_scores", "select_outliers", "fold_weight",
     "dual_branch_product", "pack_weight", "f32_to_bf16_bits", "gelu_bf16",
     "col_absmax", "dequant_mxfp4", "prep_activation", "calibrate",
-    "mxfp4_quantize_blocks", "_pad_cols", "smooth_activation")}
+    "mxfp4_quantize_blocks", "_pad_cols", "smooth_activation", "search_layer")}
 
 
 def _e2m1_ties_away(q):
@@ -345,7 +345,37 @@ def _smoothing_accepts_nonfinite(act_scale, w_scale, alpha):
     return s, inv_s
 
 
+def _search_with(metric, key):
+    """search_layer with another error metric or tie rule."""
+    def search(X, W, alphas, ks, layouts=(orc.LAYOUT_32x1,), X_eval=None):
+        Xe = X if X_eval is None else X_eval
+        exact = Xe.astype(np.float64) @ W.astype(np.float64).T
+        errors = {}
+        for layout in layouts:
+            for k in ks:
+                for alpha in alphas:
+                    c = orc.calibrate(X, W, alpha, k)
+                    pw = orc.pack_weight(W, c["s"], c["O"], c["J"], layout)
+                    pa = orc.prep_activation(Xe, c["inv_s"], c["O"], c["J"])
+                    Y = orc.dual_branch_product(pa["aq"], pa["sfa"], pa["xo"], pw["wq"], pw["sfb"],
+                                                pw["w_hp"])
+                    errors[(alpha, k, layout)] = metric(Y, exact)
+        return min(errors, key=lambda cnd: key(errors[cnd], cnd)), errors
+    return search
+
+
+_frob_rel = lambda Y, E: float(np.sqrt(np.sum((Y - E) ** 2) / np.sum(E * E)))
+_search_unnormalised = _search_with(lambda Y, E: float(np.sqrt(np.sum((Y - E) ** 2))),
+                                    lambda e, c: (e, c[1]))
+_search_no_sqrt = _search_with(lambda Y, E: float(np.sum((Y - E) ** 2) / np.sum(E * E)),
+                               lambda e, c: (e, c[1]))
+_search_ties_larger_k = _search_with(_frob_rel, lambda e, c: (e, -c[1]))
+
+
 MUTANTS = {
+    "search_unnormalised": {"search_layer": _search_unnormalised},
+    "search_no_sqrt": {"search_layer": _search_no_sqrt},
+    "search_ties_larger_k": {"search_layer": _search_ties_larger_k},
     "block_amax_ignores_nan": {"mxfp4_quantize_blocks": _block_amax_ignores_nan},
     "exponent_inf_126": {"mx_shared_exponent": _exponent_inf_126},
     "dequant_nan_scale_finite": {"dequant_mxfp4": _dequant_nan_scale_finite},

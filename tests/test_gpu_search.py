@@ -47,3 +47,20 @@ def test_relative_error_kernel():
     ref = ((Y.double() - R.double()).pow(2).sum() / R.double().pow(2).sum()).sqrt().item()
     assert abs(e - ref) <= 1e-9 * max(1.0, ref)
     assert tuning.relative_error(R.to(torch.bfloat16)[:0], R[:0]) == 0.0
+
+
+def test_search_hand_worked_case():
+    """The hand-worked case of tests/golden/search_layer_hand.txt on the GPU:
+    every quantised product there is exact in bf16 and the reference product
+    is exact in float32, so the library's errors are the hand values."""
+    from tests import search_hand_case as hc
+    X, W = hc.inputs()
+    Xg = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    Wg = torch.from_numpy(W).to(torch.bfloat16).cuda()
+    res = tuning.search_layer(Xg, Wg, hc.ALPHAS, hc.KS)
+    assert w4.last_error()[0] == w4.OK
+    table, best = hc.expected()
+    assert set(res.errors) == set(table)
+    for c, e in table.items():
+        assert abs(res.errors[c] - e) <= 1e-12, (c, res.errors[c], e)
+    assert res.best == best

@@ -414,3 +414,16 @@ def test_calibration_refuses_non_finite_magnitudes():
                 orc.smoothing_factors(aa, ww, 0.5)
     s, inv_s = orc.smoothing_factors(a, w, 0.5)
     assert (s == 1).all() and (inv_s == 1).all()
+
+
+def test_search_layer_hand_worked():
+    """The relative Frobenius metric and the tie rule on a case whose every
+    candidate was worked by hand (tests/golden/search_layer_hand.txt)."""
+    from tests import search_hand_case as hc
+    X, W = hc.inputs()
+    table, best_hand = hc.expected()
+    best, err = orc.search_layer(X, W, hc.ALPHAS, hc.KS)
+    assert set(err) == set(table)
+    for c, e in table.items():
+        assert abs(err[c] - e) <= 1e-12, (c, err[c], e)
+    assert best == best_hand

@@ -6,12 +6,14 @@ shallow and deep layers as the next step, without a procedure.  The plainest
 one, used here: run the whole quantised layer for every candidate on
 calibration activations and keep the candidate with the smallest relative
 Frobenius error ||Y - X W^T|| / ||X W^T||, preferring the smaller k (the
-high-precision budget) on ties.
+high-precision budget) on ties, then the candidate listed first (layouts,
+then k, then alpha, in the order given).
 
 Every candidate runs through the library: calib_observe once (the absmax
 statistics do not depend on alpha or k), then calib_finalize, pack_weight,
 linear and error_sums per candidate.  The reference product X W^T is a plain
-float32 cuBLAS GEMM (torch.matmul).
+float32 cuBLAS GEMM (torch.matmul): an evaluation-only reference for scoring
+candidates, not a step of the quantised layer.
 """
 from __future__ import annotations
 

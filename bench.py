@@ -1,6 +1,6 @@
 """Benchmark of the W4A4 dual-branch linear on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--report]
                     [--workload full|full_up|full_down|mid_up|mid_down|ffn0|ffn2|tiny|sweep
                                 |ffn|ffn_mid]
 
@@ -19,12 +19,22 @@ rate).  Per-kernel numbers come from CUDA events recorded on the launching
 stream around each launch inside the timed region.  The full workload's
 inputs are larger than L2 (X is 590 MB / 1.59 GB), so nothing is flushed;
 where a step's inputs are under twice the L2 size a 256 MB buffer is written
-between steps, outside each step's own events.  ``e2e`` repeats the step
-from pinned host buffers with the copies inside the timed region.
+between steps, outside each step's own events.  ``e2e`` times the online
+layer through the library's host-buffer call (w4a4_linear_host: upload of X,
+prep, GEMM, download of Y in one call per layer), with the copies inside the
+timed region; the offline half's device time is reported beside it.
 
-Under torchrun each rank runs the same per-GPU workload on its own token
-shard (weak scaling, no collective on the data path); the step time is the
-max over ranks, ``value`` counts the work of all ranks.
+``--gpus N`` runs N ranks, one per GPU: launched without a launcher around it,
+bench.py starts them itself through torch's launcher (rendezvous on
+127.0.0.1); under torchrun it runs as the rank it is given.  Each rank runs
+the same per-GPU workload on its own token shard (weak scaling, no collective
+on the data path); the step time is the max over ranks, ``value`` counts the
+work of all ranks.
+
+``--report`` prints one JSON line per configuration (tiny, ffn.0, ffn.2, the
+two full layers, every sweep point) with the GEMM's TFLOPS and fraction of
+peak, the prep kernel's GB/s, the SNR of Y against the unquantised float64
+X W^T, a cuBLAS bf16 GEMM of the same shape and the oracle on a sample.
 
 ``--impl reference`` times the CPU oracle (the numpy reference the tests
 check the GPU against) on a bounded row sample of the same workload, on
@@ -272,8 +282,7 @@ class ClockSampler:
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
 # gemm_dual_pair_kernel on the "full" workload (mean of the up and down
-# launches), from one ncu capture of this bench (summary and command in
-# profiles/gemm_dual_pair_traffic_full_T57600.md).  Valid only for the GEMM
+# launches), from one ncu capture of this bench.  Valid only for the GEMM
 # sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
 # for any other source or workload.
 GEMM_TRAFFIC = {
@@ -365,6 +374,16 @@ class LayerRun:
         return 2
 
 
+def check_device(local: int):
+    """One rank per GPU: a rank whose local index has no GPU stops here (two
+    ranks on one GPU are not run)."""
+    import torch
+    n = torch.cuda.device_count()
+    if local >= n:
+        raise SystemExit(f"bench.py: rank with LOCAL_RANK={local} has no GPU "
+                         f"({n} visible); run at most {n} ranks")
+
+
 def cublas_bf16_context(runs, reps=5):
     """cuBLAS bf16 GEMM of the same shapes (Y = X W^T through torch.mm), timed
     after the timed region as context: the unquantised product this path
@@ -394,6 +413,7 @@ def run_gpu(args):
     import w4a4_mxfp4_outlier_b200 as w4
 
     world, rank, local = dist_env()
+    check_device(local)
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     active = dist_init("nccl", world, rank)
@@ -453,6 +473,8 @@ def run_gpu(args):
                for i in range(len(runs))]
     calib_ms = [sum(e[i]["off"][0].elapsed_time(e[i]["off"][1]) for e in evs) / args.steps
                 for i in range(len(runs))]
+    offline_ms = [sum(e[i]["off"][0].elapsed_time(e[i]["on"][0]) for e in evs) / args.steps
+                  for i in range(len(runs))]
     gemm_tflops = flops / (sum(gemm_ms) * 1e-3) / 1e12
     prep_bytes = sum(layer_bytes_prep(r.L, r.d) for r in runs)
     prep_gbs = prep_bytes / (sum(prep_ms) * 1e-3) / 1e9
@@ -475,6 +497,8 @@ def run_gpu(args):
 
     cublas_ms = cublas_bf16_context(runs)
     e2e = run_e2e(args, runs, w4, device, active) if not args.no_e2e else None
+    if e2e is not None:
+        e2e["offline_ms"] = [round(x, 4) for x in offline_ms]
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(layers, runs, rows=256, outs=1024)
@@ -517,66 +541,64 @@ def run_gpu(args):
 
 
 def run_e2e(args, runs, w4, device, active):
-    """Same step through the public calls with host buffers: every step copies
-    X and W of each layer from pinned host memory, runs the whole path and
-    copies Y back, on three streams (uploads, compute, downloads; PCIe is
-    full duplex).  A layer's compute waits only for its own inputs and for
-    the previous step's download of its Y; its download waits only for its
-    compute; the next step's upload of its X and W waits only for this
-    step's compute of that layer to have read them.  So consecutive steps
-    pipeline: the uploads run back to back and set the pace."""
+    """The online layer end to end through the library's host-buffer call,
+    w4a4_linear_host: each call copies X from pinned host memory to the
+    device, runs the activation prep and the dual-branch GEMM, and copies Y
+    back to pinned host memory, all enqueued by the library on the stream it
+    is given.  A step is one such call per layer of the workload.  Two buffer
+    sets per layer on two streams alternate between consecutive steps, so one
+    step's uploads overlap the previous step's compute and downloads (PCIe is
+    full duplex).  The offline half (calibration and pack, once per layer in
+    deployment) ran before the timed region; its device time is in the main
+    line's kernels (calib_absmax_ms) and in offline_ms below."""
     import torch
-    hosts = []
+    sets = []
     for r in runs:
-        hosts.append((r.X.cpu().pin_memory(), r.W.cpu().pin_memory(),
-                      torch.empty(r.Y.shape, dtype=r.Y.dtype).pin_memory()))
-    h2d = sum(x.numel() * 2 + w.numel() * 2 for x, w, _ in hosts)
-    d2h = sum(y.numel() * 2 for _, _, y in hosts)
+        xh = r.X.cpu().pin_memory()
+        per = []
+        for _ in range(2):
+            per.append({"xd": torch.empty_like(r.X), "yd": torch.empty_like(r.Y),
+                        "yh": torch.empty(r.Y.shape, dtype=r.Y.dtype).pin_memory(),
+                        "ws": torch.empty(w4.workspace_size(r.L.T, r.L.d_in, r.L.d_out, r.L.k),
+                                          dtype=torch.uint8, device=device),
+                        "stream": torch.cuda.Stream(device)})
+        sets.append((xh, per))
+    h2d = sum(r.L.T * r.L.d_in * 2 for r in runs)
+    d2h = sum(r.L.T * r.L.d_out * 2 for r in runs)
     steps = max(3, min(args.steps, 8))
-    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    prev_c = [None] * len(runs)     # per layer: the previous step's compute is done
-    prev_o = [None] * len(runs)     # per layer: the previous step's download is done
+    calls = [0]
 
-    def step():
-        for i, (r, (xh, wh, yh)) in enumerate(zip(runs, hosts)):
-            if prev_c[i] is not None:
-                s_in.wait_event(prev_c[i])          # X and W are no longer read
-            with torch.cuda.stream(s_in):
-                r.X.copy_(xh, non_blocking=True)
-                r.W.copy_(wh, non_blocking=True)
-                e_in = torch.cuda.Event()
-                e_in.record(s_in)
-            s_comp.wait_event(e_in)
-            if prev_o[i] is not None:
-                s_comp.wait_event(prev_o[i])        # Y has been read out
-            with torch.cuda.stream(s_comp):
-                r.offline()
-                r.online()
-                e_c = torch.cuda.Event()
-                e_c.record(s_comp)
-            s_out.wait_event(e_c)
-            with torch.cuda.stream(s_out):
-                yh.copy_(r.Y, non_blocking=True)
-                e_o = torch.cuda.Event()
-                e_o.record(s_out)
-            prev_c[i], prev_o[i] = e_c, e_o
+    def step(k):
+        for r, (xh, per) in zip(runs, sets):
+            b = per[k % 2]
+            w4.linear_host(xh, r.pw, b["xd"], b["ws"], b["yd"], b["yh"], stream=b["stream"])
+            calls[0] += 1
 
-    def join():
-        # every step's results are on the host
-        s_in.wait_stream(s_comp)
-        s_in.wait_stream(s_out)
+    def join(s):
+        for _, per in sets:
+            for b in per:
+                s.wait_stream(b["stream"])
 
-    step()
-    join()
+    main_s = torch.cuda.current_stream(device)
+    step(0)
+    step(1)
     torch.cuda.synchronize()
+    # the step's Y arrived on the host, bit for bit what the device path gives
+    for r, (_, per) in zip(runs, sets):
+        if not torch.equal(per[1]["yh"], r.Y.cpu()):
+            raise RuntimeError(f"{r.L.name}: linear_host output differs from the device path")
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     dist_barrier(active, device)
-    t0.record(s_in)
-    for _ in range(steps):
-        step()
-    join()
-    t1.record(s_in)
+    t0.record(main_s)
+    for _, per in sets:
+        for b in per:
+            b["stream"].wait_stream(main_s)
+    calls[0] = 0
+    for k in range(steps):
+        step(k)
+    join(main_s)
+    t1.record(main_s)
     torch.cuda.synchronize()
     ms = dist_max(t0.elapsed_time(t1) / steps, active, device)
     world = dist_env()[0]
@@ -585,9 +607,13 @@ def run_e2e(args, runs, w4, device, active):
             "ms_per_step": round(ms, 3), "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "h2d_gbs": round(h2d / (ms * 1e-3) / 1e9, 1),
-            "overlap": "uploads, compute and downloads on three streams; consecutive steps "
-                       "pipelined (the timed region runs from the first upload to the last "
-                       "download)"}
+            "d2h_gbs": round(d2h / (ms * 1e-3) / 1e9, 1),
+            "path": "w4a4_linear_host per layer and step (H2D of X, prep, dual GEMM, D2H of Y, "
+                    "all enqueued by the library), two buffer sets per layer on alternating "
+                    "streams",
+            "calls_per_step": calls[0] // steps,
+            "offline": "calibration and pack once per layer before the timed region "
+                       "(device time reported as offline_ms)"}
 
 
 # ---------------------------------------------------------------------------
@@ -704,6 +730,93 @@ def ffn_workload_config(workload, Lu, Ld, world, flushed=None):
                     "+ down GEMM (packed weights prepared before timing)"}
 
 
+def report_layers():
+    """The configurations of the report: tiny, ffn.0 and ffn.2 at T = 4096,
+    the two layers of the full T = 57600 workload, every sweep point."""
+    import synth
+    return ([synth.TINY, synth.FFN0, synth.FFN2, synth.FULL_UP, synth.FULL_DOWN]
+            + synth.sweep_layers())
+
+
+def snr_db(Y, Y_exact) -> float:
+    """10 log10(sum Y_exact^2 / sum (Y - Y_exact)^2)."""
+    import numpy as np
+    num = float(np.sum(Y_exact * Y_exact))
+    den = float(np.sum((Y - Y_exact) ** 2))
+    return 10.0 * np.log10(num / den) if den > 0 else float("inf")
+
+
+def run_report(args):
+    """One JSON line per configuration: the dual GEMM's TFLOPS and fraction of
+    the FP4 peak, the prep kernel's GB/s and fraction of the HBM copy
+    bandwidth, the SNR of Y against the unquantised float64 X W^T on sampled
+    rows (reported, not a pass criterion), a cuBLAS bf16 GEMM of the same
+    shape as context, and the CPU oracle on a row sample.  Single GPU."""
+    import numpy as np
+    import torch
+
+    import synth
+    import w4a4_mxfp4_outlier_b200 as w4
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("bench.py --report runs on one GPU")
+    check_device(local)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    peaks, src = measured_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    for L in report_layers():
+        r = LayerRun(L, device, w4, synth)
+        for _ in range(args.warmup):
+            r.offline()
+            r.online()
+        flush = l2_flush_buffer(layer_input_bytes(L), device)
+        evs = [[mk(), mk(), mk()] for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            r.offline()
+            if flush is not None:
+                flush.zero_()
+            r.online(evs[k])
+        torch.cuda.synchronize()
+        st, bits = w4.last_error()
+        if st != w4.OK:
+            raise RuntimeError(f"{L.name}: device error word {bits:#x}")
+        gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+        prep_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        gemm_tflops = L.flops / (gemm_ms * 1e-3) / 1e12
+        prep_gbs = layer_bytes_prep(L, r.d) / (prep_ms * 1e-3) / 1e9
+        rows = synth.sample_rows(L.T, 256)
+        ridx = rows.to(device)
+        Xr = r.X[ridx].double().cpu().numpy()
+        exact = Xr @ r.W.double().cpu().numpy().T
+        snr = snr_db(r.Y[ridx].double().cpu().numpy(), exact)
+        cub_ms = cublas_bf16_context([r])[0]
+        Xs, Ws = _host_samples([L], [r], 64, 256)
+        of, osec = oracle_sample([L], 64, 256, Xs, Ws)
+        out = {"report": L.name,
+               "config": f"T={L.T} {L.d_in}->{L.d_out} k={L.k} alpha={L.alpha} "
+                         f"{LAYOUT_NAMES[L.layout]}",
+               "steps": args.steps, "warmup": args.warmup, "l2": l2_note(flush is not None),
+               "gemm_ms": round(gemm_ms, 4), "gemm_tflops": round(gemm_tflops, 1),
+               "gemm_frac_fp4_peak": round(gemm_tflops / fp4_peak, 4),
+               "gemm_frac_fp4_nominal_9pf": round(gemm_tflops / FP4_NOMINAL_TFLOPS, 4),
+               "fp4_peak": f"{src} bf16_tflops x {FP4_PER_BF16:g} = {fp4_peak:.1f} TFLOP/s",
+               "prep_ms": round(prep_ms, 4), "prep_gbs": round(prep_gbs, 1),
+               "prep_frac_hbm_measured": round(prep_gbs / peaks["hbm_gbs"], 4),
+               "prep_frac_hbm_nominal_8tbs": round(prep_gbs / HBM_NOMINAL_GBS, 4),
+               "snr_db_vs_fp64_xw": round(snr, 2), "snr_rows": int(rows.numel()),
+               "cublas_bf16_ms": round(cub_ms, 4),
+               "cublas_bf16_tflops": round(L.flops / (cub_ms * 1e-3) / 1e12, 1),
+               "oracle": {"seconds": round(osec, 2), "tflops": round(of / osec / 1e12, 8),
+                          "cores": _threads_used(),
+                          "sample": "64 token rows x 256 output channels, whole path in numpy"}}
+        print(json.dumps(out), flush=True)
+        del r, flush, Xr, exact
+        torch.cuda.empty_cache()
+
+
 def run_reference(args):
     import synth
     world, rank, _ = dist_env()
@@ -756,6 +869,7 @@ def run_ffn(args):
     from w4a4_mxfp4_outlier_b200 import ffn
 
     world, rank, local = dist_env()
+    check_device(local)
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     active = dist_init("nccl", world, rank)
@@ -867,7 +981,26 @@ def run_ffn(args):
         dist.destroy_process_group()
 
 
+def free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def self_launch_cmd(argv, n: int, port: int):
+    """The command that runs this script on n ranks of one node: torch's own
+    launcher (one process per GPU, RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*
+    set for each), rendezvous on 127.0.0.1, the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -878,15 +1011,29 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--report", action="store_true",
+                    help="one JSON line per workload configuration (tiny, ffn0, ffn2, the two "
+                         "full layers, every sweep point) instead of the headline line")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least three untimed warm-up steps
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # launched as `bench.py --gpus N`: start the N ranks here, one per GPU,
+        # and return the launcher's status (each rank re-enters with WORLD_SIZE set)
+        return subprocess.call(self_launch_cmd(argv, args.gpus, free_port()))
+    world = dist_env()[0]
+    if world != args.gpus and world > 1:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; running {world} ranks",
+              file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.report:
+        run_report(args)
     elif args.workload in ("ffn", "ffn_mid"):
         run_ffn(args)
     else:
         run_gpu(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

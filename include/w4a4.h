@@ -365,6 +365,19 @@ w4a4_status w4a4_error_sums(const void* Y, int64_t ldy, const float* Yref, int64
  * error word.  clear != 0 resets the word. */
 w4a4_status w4a4_last_error(void* stream, int clear, uint32_t* bits);
 
+/* Failure-detection test hook, not for production use.  Sets, on the current
+ * device, how long a device pipeline wait may last before it is abandoned
+ * (wait_limit_ns; 0 restores the default of about 2 s; at most the default)
+ * and a fault mask: W4A4_FAULT_PREP_SKIP_LOADS makes the activation-prep
+ * kernel's producer issue no row copies, so every consumer wait of the next
+ * prep launches runs out -- the kernel records W4A4_ERR_TIMEOUT in the device
+ * error word and returns, leaving its outputs incomplete, with no trap and the
+ * context usable.  Synchronises the device first.  Call with (0, 0) to
+ * restore normal operation.  INVALID_ARG for an unknown mask bit or a limit
+ * above the default. */
+#define W4A4_FAULT_PREP_SKIP_LOADS 1u
+w4a4_status w4a4_test_fault(uint32_t mask, uint64_t wait_limit_ns);
+
 /* Number of streaming multiprocessors of the current device (used to size
  * persistent grids); 0 on error. */
 int w4a4_num_sms(void);

@@ -252,3 +252,10 @@ def test_binding_rejects_what_is_not_bf16_rows():
     with pytest.raises(w4.W4A4Error) as e:
         w4._rows_bf16(X, "x")                           # host memory where device rows are read
     assert e.value.status == w4.ERR_INVALID_ARG
+
+
+def test_fault_hook_validates_before_touching_the_device():
+    # unknown mask bits and limits above the default are refused before any CUDA call
+    assert w4._test_fault(2, 0) == w4.ERR_INVALID_ARG
+    assert w4._test_fault(1, 3_000_000_000) == w4.ERR_INVALID_ARG
+    assert "inf or NaN" in w4.status_string(w4.ERR_NONFINITE_CALIB)

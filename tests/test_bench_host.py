@@ -148,3 +148,29 @@ def test_clock_sampler_without_nvml_or_nvidia_smi():
     s.mark_end()
     out = s.stop()
     assert out["sm_mhz"] is None and out["reasons"]
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` (no launcher around it) starts two ranks itself;
+    rank 0 alone prints the one JSON line, which reports both ranks.  The
+    reference arm runs here (CPU), through the same launch path."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        "--gpus", "2", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "0"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_self_launch_command():
+    cmd = bench.self_launch_cmd(["--gpus", "4", "--steps", "5"], 4, 29512)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert "--master-port=29512" in cmd and cmd[-4:] == ["--gpus", "4", "--steps", "5"]
+    assert cmd[-5].endswith("bench.py")

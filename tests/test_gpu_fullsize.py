@@ -95,15 +95,22 @@ def test_full_size_ffn_sampled():
     gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, "ffn_full_down")
 
 
-SWEEP_EXTREMES = [L for L in synth.sweep_layers()
-                  if (L.k, L.layout, L.alpha) in ((0, 1, 0.5), (256, 1, 0.5), (16, 2, 0.7), (256, 2, 0.7))]
+def _channel_groups(d_out: int, n_groups: int, seed: int = 9) -> np.ndarray:
+    """Whole 32-row groups of output channels (so 32x32 weight tiles sampled
+    this way are the tiles of the full pack), seeded."""
+    g = np.sort(np.random.default_rng(seed).choice(d_out // 32, n_groups, replace=False))
+    return (g[:, None] * 32 + np.arange(32)[None, :]).reshape(-1)
 
 
-@pytest.mark.parametrize("L", SWEEP_EXTREMES, ids=lambda L: L.name)
+@pytest.mark.parametrize("L", synth.sweep_layers(), ids=lambda L: L.name)
 def test_sweep_sampled(L):
-    """Sweep points at their own size (T = 16384, 5120 -> 13824) with the
-    32x32-tile and 128x1-stripe weight scales and the smallest and largest k:
-    the packed weight in full, codes and Y on 512 sampled token rows."""
+    """Every sweep point at its own size (T = 16384, 5120 -> 13824): k in
+    {0, 16, 64, 256} x weight scales {32x1, 32x32, 128x1} x alpha in {0.5, 0.7}
+    in bench.py's launch configuration (calibration, pack, prep and GEMM on the
+    whole tensors).  Checked on what the oracle affords: the outlier set, the
+    packed weight of 16 whole 32-channel groups (512 output channels), the
+    activation codes of 512 sampled token rows, and Y on those rows and
+    channels."""
     X, W = gu.gen(L)
     pw = w4.calibrate(X, W, L.alpha, L.k, L.layout)
     act = w4.alloc_act(L.T, pw)
@@ -114,16 +121,20 @@ def test_sweep_sampled(L):
     assert st == w4.OK, f"device error word {bits:#x}"
     c = gu.oracle_calib_from_gpu(pw)
     np.testing.assert_array_equal(pw.O.cpu().numpy(), c["O"])
-    ref_w = orc.pack_weight(gu.to_np_f32(W), c["s"], c["O"], c["J"], L.layout)
+
+    chans = _channel_groups(L.d_out, 16)
+    cidx = torch.from_numpy(chans).cuda()
+    ref_w = orc.pack_weight(gu.to_np_f32(W[cidx]), c["s"], c["O"], c["J"], L.layout)
     d = pw.dims
     nb = ref_w["sfb"].shape[1]
-    np.testing.assert_array_equal(pw.wq.view(L.d_out, -1).cpu().numpy()[:, :nb * 16], ref_w["wq"])
+    np.testing.assert_array_equal(pw.wq.view(L.d_out, -1)[cidx].cpu().numpy()[:, :nb * 16],
+                                  ref_w["wq"])
     if d.nblk:
-        sfb = gu.sf_canonical(pw.sfb, d.sfb_rows, d.nblk, nb)
-        np.testing.assert_array_equal(sfb[:L.d_out, :nb], ref_w["sfb"])
+        sfb = gu.sf_canonical(pw.sfb, chans, d.nblk, nb)
+        np.testing.assert_array_equal(sfb[:, :nb], ref_w["sfb"])
     if L.k:
-        np.testing.assert_array_equal(gu.bf16_bits(pw.w_hp).reshape(L.d_out, d.k_pad)[:, :L.k],
-                                      ref_w["w_hp"])
+        np.testing.assert_array_equal(
+            gu.bf16_bits(pw.w_hp).reshape(L.d_out, d.k_pad)[chans, :L.k], ref_w["w_hp"])
 
     rows = synth.sample_rows(L.T, 512).numpy()
     ridx = torch.from_numpy(rows).cuda()
@@ -136,4 +147,5 @@ def test_sweep_sampled(L):
         np.testing.assert_array_equal(gu.bf16_bits(act.xo[ridx])[:, :L.k], ref_a["xo"])
     Y_ref = orc.dual_branch_product(ref_a["aq"], ref_a["sfa"], ref_a["xo"], ref_w["wq"],
                                     ref_w["sfb"], ref_w["w_hp"])
-    gu.check_tolerance(gu.to_np_f32(Y[ridx]).astype(np.float64), Y_ref, L.name)
+    Ys = gu.to_np_f32(Y[ridx][:, cidx]).astype(np.float64)
+    gu.check_tolerance(Ys, Y_ref, L.name)

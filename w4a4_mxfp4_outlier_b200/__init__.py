@@ -95,6 +95,8 @@ _gemm_dual_act = _sig("w4a4_gemm_dual_act", _st, _vp, _vp, _vp, _i64, ctypes.POI
                       ctypes.POINTER(PackedWeightC), _vp, _vp, _vp, _vp, _vp)
 _error_sums = _sig("w4a4_error_sums", _st, _vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp)
 _last_error = _sig("w4a4_last_error", _st, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32))
+_test_fault = _sig("w4a4_test_fault", _st, ctypes.c_uint32, ctypes.c_uint64)
+FAULT_PREP_SKIP_LOADS = 1           # W4A4_FAULT_PREP_SKIP_LOADS
 
 EXPORTED = [
     "w4a4_abi_version", "w4a4_status_string", "w4a4_num_sms", "w4a4_get_dims",
@@ -103,7 +105,7 @@ EXPORTED = [
     "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
     "w4a4_packed_image_size", "w4a4_packed_save", "w4a4_packed_image_info", "w4a4_packed_load",
     "w4a4_error_sums", "w4a4_gelu_bf16", "w4a4_ffn_link", "w4a4_pack_weight_rows", "w4a4_permute_packed_rows",
-    "w4a4_gemm_dual_act",
+    "w4a4_gemm_dual_act", "w4a4_test_fault",
 ]
 
 
@@ -364,6 +366,13 @@ def save_packed(pw: PackedWeight, path: str, stream=None):
 def load_packed(path: str, device="cuda", stream=None) -> PackedWeight:
     with open(path, "rb") as f:
         return packed_from_bytes(f.read(), device, stream)
+
+
+def test_fault(mask: int, wait_limit_ns: int = 0):
+    """Failure-detection test hook (w4a4_test_fault): shorten the device wait
+    limit and make the prep producer skip its copies; test_fault(0, 0)
+    restores normal operation."""
+    _check(_test_fault(mask, wait_limit_ns), "test_fault")
 
 
 def last_error(clear: bool = True, stream=None):

@@ -88,10 +88,12 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
     const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
     const uint16_t* src = X + static_cast<int64_t>(blockIdx.x) * ldx;
     const int64_t src_step = static_cast<int64_t>(gridDim.x) * ldx;
+    // failure-detection test hook: no copies at all, the consumers' waits run out
+    const bool skip = (g_fault_mask & FAULT_PREP_SKIP_LOADS) != 0u;
     int64_t issued = 0;
     int u = 0;
     uint32_t ph = 0;
-    for (int64_t i = 0; i < nrows; ++i) {
+    for (int64_t i = 0; i < nrows && !skip; ++i) {
       if (i >= kPrepStages &&
           !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
         break;

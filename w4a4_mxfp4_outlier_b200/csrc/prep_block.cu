@@ -85,10 +85,12 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   if (warp == 0) {
     // ---------------- producer (whole warp; one elected lane issues) ----------------
     const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
+    // failure-detection test hook: no copies at all, the consumers' waits run out
+    const bool skip = (g_fault_mask & FAULT_PREP_SKIP_LOADS) != 0u;
     int64_t issued = 0;
     int u = 0;
     uint32_t ph = 0;
-    for (int64_t i = 0; i < nrows; ++i) {
+    for (int64_t i = 0; i < nrows && !skip; ++i) {
       if (i >= R::kSlots &&
           !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
         break;

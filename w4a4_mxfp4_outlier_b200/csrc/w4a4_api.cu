@@ -283,6 +283,18 @@ w4a4_status w4a4_linear_host(const void* X_host, int64_t T, const w4a4_packed_we
   return from_cuda(e);
 }
 
+w4a4_status w4a4_test_fault(uint32_t mask, uint64_t wait_limit_ns) {
+  if ((mask & ~static_cast<uint32_t>(FAULT_PREP_SKIP_LOADS)) != 0u) return W4A4_ERR_INVALID_ARG;
+  const uint64_t limit = wait_limit_ns == 0 ? kWaitLimitNs : wait_limit_ns;
+  if (limit > kWaitLimitNs) return W4A4_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  e = cudaMemcpyToSymbol(g_wait_limit_ns, &limit, sizeof(limit));
+  if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  e = cudaMemcpyToSymbol(g_fault_mask, &mask, sizeof(mask));
+  return from_cuda(e);
+}
+
 w4a4_status w4a4_last_error(void* stream, int clear, uint32_t* bits) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return W4A4_ERR_CUDA;

@@ -26,8 +26,16 @@ enum : uint32_t {
 // single definition is the word every kernel and the host accessor use.
 static __device__ uint32_t g_device_error = 0u;
 
-// About 2 s of wall time on %globaltimer before a wait is abandoned.
+// Wall time on %globaltimer before a wait is abandoned: about 2 s, unless a
+// failure-detection test shortened it (w4a4_test_fault).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+static __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+
+// Failure-detection test hook (w4a4_test_fault): while bit 0 is set, the
+// activation-prep producer issues no row copies, so its consumers' waits run
+// out.  Zero in normal use.
+enum : uint32_t { FAULT_PREP_SKIP_LOADS = 1u << 0 };
+static __device__ uint32_t g_fault_mask = 0u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -73,8 +81,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, or as soon as *abort becomes non-zero (another role gave up):
-// returns false then, after recording `err_bit` in the device error word.
+// g_wait_limit_ns, or as soon as *abort becomes non-zero (another role gave
+// up): returns false then, after recording `err_bit` in the device error word.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile uint32_t* abort, uint32_t err_bit) {
   const uint32_t a = smem_u32(bar);
@@ -84,7 +92,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > *static_cast<volatile uint64_t*>(&g_wait_limit_ns)) {
         atomicOr(&g_device_error, err_bit);
         if (abort != nullptr) *abort = 1u;
         return false;

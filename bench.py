@@ -773,13 +773,19 @@ def run_report(args):
             r.online()
         flush = l2_flush_buffer(layer_input_bytes(L), device)
         evs = [[mk(), mk(), mk()] for _ in range(args.steps)]
+        clocks = clock_sampler(local)
         torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.05)
+        clocks.mark_start()
         for k in range(args.steps):
             r.offline()
             if flush is not None:
                 flush.zero_()
             r.online(evs[k])
         torch.cuda.synchronize()
+        clocks.mark_end()
+        clock_info = clocks.stop()
         st, bits = w4.last_error()
         if st != w4.OK:
             raise RuntimeError(f"{L.name}: device error word {bits:#x}")
@@ -809,6 +815,7 @@ def run_report(args):
                "snr_db_vs_fp64_xw": round(snr, 2), "snr_rows": int(rows.numel()),
                "cublas_bf16_ms": round(cub_ms, 4),
                "cublas_bf16_tflops": round(L.flops / (cub_ms * 1e-3) / 1e12, 1),
+               "clocks": clock_info,
                "oracle": {"seconds": round(osec, 2), "tflops": round(of / osec / 1e12, 8),
                           "cores": _threads_used(),
                           "sample": "64 token rows x 256 output channels, whole path in numpy"}}

@@ -138,3 +138,39 @@ def test_fused_epilogue_matches_oracle_and_unfused(case):
     assert not xo[:, k_down:].any()
     # and the whole FFN: fused == unfused, bit for bit
     assert torch.equal(Y_f.view(torch.int16), Y_u.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# The down layer's Y against an oracle chain that starts from X
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("case", [(300, 512, 1376, 8, 19, 0), (300, 512, 1376, 8, 19, 1)],
+                         ids=lambda c: "T%d_%dx%d_k%d_%d_l%d" % c)
+def test_ffn_down_output_against_oracle_chain_from_x(case):
+    """Y of the whole fused FFN against the oracle run from X alone (its own
+    up product in float64, GELU, down prep, down product), with the
+    library's calibration (s, O, J) on both layers.  The GPU's bf16 Y_up may
+    lie anywhere within the up layer's tolerance of the oracle's; that band,
+    rounded outward to bf16, is carried through GELU, the smoothing multiply,
+    the MXFP4 quantiser and the down product (tests/ffn_bounds.py), giving for
+    each output an interval that contains every down product such a Y_up can
+    produce.  The GPU's Y must lie within the down layer's tolerance of that
+    interval."""
+    from tests import ffn_bounds as fb
+    T, d_model, d_ff, k_up, k_down, layout = case
+    X, W_up, W_down, f = _make_ffn(*case)
+    Y = torch.empty((T, d_model), dtype=torch.bfloat16, device="cuda")
+    ffn.forward(X, f, Y)
+    assert w4.last_error()[0] == w4.OK
+    cu, cd = gu.oracle_calib_from_gpu(f.up_plain), gu.oracle_calib_from_gpu(f.down)
+    wu = orc.pack_weight(gu.to_np_f32(W_up), cu["s"], cu["O"], cu["J"], layout)
+    au = orc.prep_activation(gu.to_np_f32(X), cu["inv_s"], cu["O"], cu["J"])
+    Yu = orc.dual_branch_product(au["aq"], au["sfa"], au["xo"], wu["wq"], wu["sfb"], wu["w_hp"])
+    Ylo, Yhi = fb.down_interval(Yu, fb.up_tolerance(Yu), cd, gu.to_np_f32(W_down), layout)
+    Yg = gu.to_np_f32(Y).astype(np.float64)
+    rms = float(np.sqrt(np.mean((0.5 * (Ylo + Yhi)) ** 2)))
+    outside = np.maximum(np.maximum(Ylo - Yg, Yg - Yhi), 0.0)
+    bound = 8e-3 * np.maximum(np.abs(Ylo), np.abs(Yhi)) + 1e-3 * rms
+    assert (outside <= bound).all(), f"{int((outside > bound).sum())} outputs outside, worst " \
+        f"{float((outside / bound).max()):.2f} of the bound"
+    # the interval says something: its typical width is a fraction of the outputs
+    assert float(np.median(Yhi - Ylo)) < 0.5 * rms

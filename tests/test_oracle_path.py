@@ -427,3 +427,35 @@ def test_search_layer_hand_worked():
     for c, e in table.items():
         assert abs(err[c] - e) <= 1e-12, (c, err[c], e)
     assert best == best_hand
+
+
+def test_ffn_chain_interval_contains_every_up_output_in_the_band():
+    """The interval the FFN chain test uses (tests/ffn_bounds.py) contains the
+    oracle's own down product for up-layer outputs drawn anywhere in the
+    band: the bound is sound (it is not a reading of the pages, it is how the
+    GPU test compares an end-to-end result with an oracle chain from X)."""
+    from tests import ffn_bounds as fb
+    rng = np.random.default_rng(0)
+    T, dm, dff = 24, 64, 160
+    q = lambda a: orc.bf16_bits_to_f32(orc.f32_to_bf16_bits(a.astype(np.float32)))
+    X = q(rng.standard_t(3, (T, dm)) * 0.3)
+    Wu, Wd = q(rng.normal(size=(dff, dm)) * 0.05), q(rng.normal(size=(dm, dff)) * 0.05)
+    cu = orc.calibrate(X, Wu, 0.6, 4)
+    wu = orc.pack_weight(Wu, cu["s"], cu["O"], cu["J"])
+    au = orc.prep_activation(X, cu["inv_s"], cu["O"], cu["J"])
+    Yu = orc.dual_branch_product(au["aq"], au["sfa"], au["xo"], wu["wq"], wu["sfb"], wu["w_hp"])
+    cd = orc.calibrate(orc.ffn_hidden(q(Yu)), Wd, 0.7, 6)
+    tol = fb.up_tolerance(Yu)
+    ylo, yhi = fb.bf16_round_out(Yu - tol, Yu + tol)
+    assert (ylo <= Yu - tol).all() and (yhi >= Yu + tol).all()
+    Ylo, Yhi = fb.down_interval(Yu, tol, cd, Wd, orc.LAYOUT_32x1)
+    wd = orc.pack_weight(Wd, cd["s"], cd["O"], cd["J"])
+    for _ in range(8):
+        yb = np.clip(q(Yu + tol * rng.uniform(-1, 1, Yu.shape)), ylo, yhi)
+        ad = orc.prep_activation(orc.ffn_hidden(yb), cd["inv_s"], cd["O"], cd["J"])
+        Yd = orc.dual_branch_product(ad["aq"], ad["sfa"], ad["xo"], wd["wq"], wd["sfb"], wd["w_hp"])
+        assert (Yd >= Ylo - 1e-9).all() and (Yd <= Yhi + 1e-9).all()
+    # and a chain that leaves the band (GELU skipped) falls outside somewhere
+    ad = orc.prep_activation(q(Yu), cd["inv_s"], cd["O"], cd["J"])
+    Yd = orc.dual_branch_product(ad["aq"], ad["sfa"], ad["xo"], wd["wq"], wd["sfb"], wd["w_hp"])
+    assert ((Yd < Ylo - 1e-9) | (Yd > Yhi + 1e-9)).any()

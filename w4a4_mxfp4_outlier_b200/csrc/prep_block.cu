@@ -11,7 +11,11 @@
 // element than prep_kernel's 8-elements-per-lane form):
 //  * a ring of rows in shared memory filled by a producer warp with bulk
 //    copies of whole rows, as in prep_kernel (its 6 slots of 32.9 KB, or 18
-//    slots of 11 KB for rows of up to 5480 elements);
+//    slots of 11 KB for rows of up to 5480 elements).  With several thread
+//    groups the producer refills whichever group's next slot is free (a
+//    non-blocking check per group) instead of waiting on the slots in ring
+//    order, where one group running behind held back the refills of the
+//    others and left them waiting for rows (up layer 0.140 -> 0.126 ms);
 //  * a group of `ntg` consumer threads handles one row, thread t the MX block
 //    t: its amax, scale and 16 code bytes need no shuffles (128x1 stripes
 //    take two, over the 4 lanes of a stripe);
@@ -87,33 +91,112 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
     const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
     // failure-detection test hook: no copies at all, the consumers' waits run out
     const bool skip = (g_fault_mask & FAULT_PREP_SKIP_LOADS) != 0u;
-    int64_t issued = 0;
-    int u = 0;
-    uint32_t ph = 0;
-    for (int64_t i = 0; i < nrows && !skip; ++i) {
-      if (i >= R::kSlots &&
-          !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
-        break;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&full[u], bytes);
-        const int64_t r = blockIdx.x + i * gridDim.x;
-        // output row r reads input row rows[r] when a row map is given
-        const uint16_t* from = X + (rows ? static_cast<int64_t>(rows[r]) : r) * ldx;
-        bulk_load(smem + static_cast<size_t>(u) * R::kSlot, from, bytes, &full[u]);
+    constexpr int G = R::kSlots / S;
+    if constexpr (G == 1) {
+      // one group owns every slot: refill them in order, blocking on each
+      int64_t issued = 0;
+      int u = 0;
+      uint32_t ph = 0;
+      for (int64_t i = 0; i < nrows && !skip; ++i) {
+        if (i >= R::kSlots &&
+            !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
+          break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full[u], bytes);
+          const int64_t r = blockIdx.x + i * gridDim.x;
+          // output row r reads input row rows[r] when a row map is given
+          const uint16_t* from = X + (rows ? static_cast<int64_t>(rows[r]) : r) * ldx;
+          bulk_load(smem + static_cast<size_t>(u) * R::kSlot, from, bytes, &full[u]);
+        }
+        __syncwarp();
+        issued = i + 1;
+        if (++u == R::kSlots) {
+          u = 0;
+          ph ^= 1u;
+        }
       }
-      __syncwarp();
-      issued = i + 1;
-      if (++u == R::kSlots) {
-        u = 0;
-        ph ^= 1u;
+      if (lane == 0 && *abort_flag) {
+        // do not leave bulk copies in flight into shared memory we give back
+        const int64_t first = issued > R::kSlots ? issued - R::kSlots : 0;
+        for (int64_t i = first; i < issued; ++i)
+          mbar_wait_bounded(&full[i % R::kSlots], static_cast<uint32_t>((i / R::kSlots) & 1),
+                            nullptr, DEVERR_TIMEOUT_PREP);
       }
-    }
-    if (lane == 0 && *abort_flag) {
-      // do not leave bulk copies in flight into shared memory we give back
-      const int64_t first = issued > R::kSlots ? issued - R::kSlots : 0;
-      for (int64_t i = first; i < issued; ++i)
-        mbar_wait_bounded(&full[i % R::kSlots], static_cast<uint32_t>((i / R::kSlots) & 1),
-                          nullptr, DEVERR_TIMEOUT_PREP);
+    } else {
+      // Rows go to the groups' slots in a fixed pattern (row i to slot i mod
+      // kSlots; group g owns slots g*S .. g*S + S - 1), and each group consumes
+      // its rows in order.  The producer refills whichever group's next slot is
+      // free, so one slow group does not hold back the others' refills.
+      int gc[G], gj[G];                       // per group: ring cycle and slot of its next row
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        gc[q] = 0;
+        gj[q] = 0;
+      }
+      uint64_t idle_since = 0;
+      bool failed = false;
+      while (!skip) {
+        bool left = false, progress = false;
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          const int64_t i = static_cast<int64_t>(R::kSlots) * gc[q] + q * S + gj[q];
+          if (i >= nrows) continue;
+          left = true;
+          const int u = q * S + gj[q];
+          bool free_slot = true;
+          if (gc[q] > 0) {
+            const uint32_t parity = static_cast<uint32_t>(gc[q] - 1) & 1u;
+            free_slot = __shfl_sync(0xFFFFFFFFu, mbar_test_wait(smem_u32(&empty[u]), parity) ? 1 : 0, 0) != 0;
+          }
+          if (!free_slot) continue;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&full[u], bytes);
+            const int64_t r = blockIdx.x + i * gridDim.x;
+            // output row r reads input row rows[r] when a row map is given
+            const uint16_t* from = X + (rows ? static_cast<int64_t>(rows[r]) : r) * ldx;
+            bulk_load(smem + static_cast<size_t>(u) * R::kSlot, from, bytes, &full[u]);
+          }
+          __syncwarp();
+          if (++gj[q] == S) {
+            gj[q] = 0;
+            ++gc[q];
+          }
+          progress = true;
+        }
+        if (!left) break;
+        if (progress) {
+          idle_since = 0;
+          continue;
+        }
+        __nanosleep(32);
+        if (*abort_flag) {
+          failed = true;
+          break;
+        }
+        const uint64_t now = globaltimer_ns();
+        if (idle_since == 0) {
+          idle_since = now;
+        } else if (now - idle_since > *static_cast<volatile uint64_t*>(&g_wait_limit_ns)) {
+          if (lane == 0) {
+            atomicOr(&g_device_error, DEVERR_TIMEOUT_PREP);
+            *abort_flag = 1u;
+          }
+          failed = true;
+          break;
+        }
+      }
+      if (lane == 0 && (failed || *abort_flag)) {
+        // do not leave bulk copies in flight into shared memory we give back:
+        // the latest fill of every slot
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+          for (int j = 0; j < S; ++j) {
+            const int fills = gc[q] + (j < gj[q] ? 1 : 0);
+            if (fills > 0)
+              mbar_wait_bounded(&full[q * S + j], static_cast<uint32_t>(fills - 1) & 1u, nullptr,
+                                DEVERR_TIMEOUT_PREP);
+          }
+      }
     }
     __syncwarp();
     return;
@@ -166,7 +249,10 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
     }
   }
   const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
-  const int64_t atoms_k = nblk >> 2;
+  // this lane's block in row 0 of the codes and of the scale atoms
+  uint8_t* const aq_lane = aq + 16 * t;
+  uint8_t* const sfa_lane = sfa + ((t >> 2) << 9) + (t & 3);
+  const uint32_t atom_row = static_cast<uint32_t>(nblk >> 2) << 9;   // bytes per 128-row atom row
   const uint32_t ws = static_cast<uint32_t>(m) >> 2;        // the rotation back: whole words ...
   const uint32_t bs = 8u * (static_cast<uint32_t>(m) & 3u);  // ... then bits
   uint32_t ph = 0;
@@ -186,7 +272,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
       }
       const uint8_t* ring = smem + j * R::kSlot;          // compile-time offset (+ gbase in go)
       const uint8_t* slot = ring + gbase;
-      const int64_t r = blockIdx.x + (i0 + u) * gridDim.x;
+      const int r = static_cast<int>(blockIdx.x + (i0 + u) * gridDim.x);   // T < 2^31
       float2 v[16];
       float amax = 0.f;
       if (enc) {
@@ -232,12 +318,13 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         }
         const uint4 out = make_uint4(__funnelshift_l(a3, a0, bs), __funnelshift_l(a0, a1, bs),
                                      __funnelshift_l(a1, a2, bs), __funnelshift_l(a2, a3, bs));
-        *reinterpret_cast<uint4*>(aq + r * aq_row + 16 * t) = out;
-        const int64_t sf_row = (((r >> 7) * atoms_k) << 9) + ((r & 31) << 4) + (((r & 127) >> 5) << 2);
-        sfa[sf_row + ((t >> 2) << 9) + (t & 3)] = static_cast<uint8_t>(code);
+        *reinterpret_cast<uint4*>(aq_lane + static_cast<int64_t>(r) * aq_row) = out;
+        const uint32_t rl = static_cast<uint32_t>(r) & 127u;
+        sfa_lane[static_cast<int64_t>(static_cast<uint32_t>(r) >> 7) * atom_row +
+                 (((rl & 31u) << 4) | ((rl >> 5) << 2))] = static_cast<uint8_t>(code);
       }
       if (t < xo_row) {
-        uint32_t* xo_p = xo + r * xo_row;
+        uint32_t* xo_p = xo + static_cast<int64_t>(r) * xo_row;
         const float x0 = pb_ring_f32(ring, oo0);
         const float x1 = pb_ring_f32(ring, oo1);
         const float2 vv = __fmul2_rn(make_float2(x0, x1), oinv);

@@ -281,14 +281,20 @@ class ClockSampler:
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
-# gemm_dual_pair_kernel on the "full" workload (mean of the up and down
-# launches), from one ncu capture of this bench.  Valid only for the GEMM
-# sources with this SHA-256 (gemm.cu then w4a4_device.cuh); reported as null
-# for any other source or workload.
+# gemm_dual_pair_kernel, from one ncu capture each of the mid-size layers
+# (T = 16384: the up layer 5120 -> 13824 and the down layer 13824 -> 5120;
+# counter captures are kept to mid-size workloads).  Every DRAM stream of the
+# GEMM grows in proportion to T (A, its scales and X_O are read once per
+# 384- or 256-column tile sweep, B once per raster group of M tiles, Y
+# written once), so a full-workload launch is the mean of the two captures
+# times 57600 / 16384.  Valid only for the GEMM sources with this SHA-256
+# (gemm.cu then w4a4_device.cuh); reported as null for any other source or
+# workload.
 GEMM_TRAFFIC = {
-    "sha256": "fdf6e8cbb15fd461000b350611761f06b41b430cae5d957ab8fb42b8306a63e9",
+    "sha256": "74f3969d5eec1afe049564ddcdb823c37113c39eb14a4580bf65b6de8ce6b578",
     "workload": "full",
-    "bytes_per_launch": (581736448 + 1551764992 + 1417102080 + 573487104) / 2,
+    "mid_bytes": {"up": 167202048 + 408370688, "down": 310143744 + 148844288},
+    "scale": 57600 / 16384,
 }
 
 
@@ -301,7 +307,8 @@ def gemm_traffic(workload: str):
             h.update(fh.read())
     if h.hexdigest() != GEMM_TRAFFIC["sha256"] or workload != GEMM_TRAFFIC["workload"]:
         return None
-    return int(GEMM_TRAFFIC["bytes_per_launch"])
+    mid = GEMM_TRAFFIC["mid_bytes"]
+    return int((mid["up"] + mid["down"]) / 2 * GEMM_TRAFFIC["scale"])
 
 
 def peak_keys(timed_seconds: float):
@@ -489,7 +496,7 @@ def run_gpu(args):
     roof = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
             "traffic": gemm_traffic(args.workload),
-            "traffic_unit": "bytes per launch (ncu dram read + write)",
+            "traffic_unit": "bytes per launch (ncu dram read + write on T=16384, scaled to T=57600)",
             "kernel": "gemm_dual_pair_kernel",
             "peak_source": f"{src}: {key} x {FP4_PER_BF16:g} (nominal FP4:BF16 ratio), of measured",
             "frac_of_other_peak": round(gemm_tflops / other, 4),

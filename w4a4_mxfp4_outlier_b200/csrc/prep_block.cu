@@ -74,7 +74,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   if (threadIdx.x == 0) {
     for (int u = 0; u < R::kSlots; ++u) {
       mbar_init(&full[u], 1);
-      mbar_init(&empty[u], ntg / 32);
+      // + the producer's outlier gather in the one-group form
+      mbar_init(&empty[u], ntg / 32 + ((R::kSlots / S == 1 && k > 0) ? 1 : 0));
     }
     *abort_flag = 0u;
     fence_barrier_init();
@@ -88,7 +89,57 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer (whole warp; one elected lane issues) ----------------
+    // The outlier columns of a row (X_O, k_pad / 2 bf16 pairs) are extra
+    // work on top of the blocks; done always by the same consumer warp they
+    // made it slower than the others, and every slot's refill waited for it.
+    // With one thread group the producer gathers them (it waits for the row
+    // to land, writes X_O, then arrives on the slot's "empty" barrier with the
+    // consumer warps): down layer 0.350 -> 0.310 ms.  With several groups the
+    // producer polls and must stay light, so the group's consumer warps take
+    // the rows' outliers in turn (row i: warp i mod warps-per-group).
     const uint32_t bytes = static_cast<uint32_t>(d_in) * 2u;
+    const int xo_pairs = k_pad >> 1;                        // bf16 pairs per row of X_O
+    // the first two pairs of this lane (p = lane, lane + 32) from registers,
+    // any further ones (k > 128) read O and inv_s again
+    uint32_t po[4];
+    float2 pinv[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int p2 = 2 * (lane + 32 * q);
+      po[2 * q] = p2 < k ? 2u * static_cast<uint32_t>(O[p2]) : R::kZero;
+      po[2 * q + 1] = p2 + 1 < k ? 2u * static_cast<uint32_t>(O[p2 + 1]) : R::kZero;
+      pinv[q] = make_float2(p2 < k ? inv_s[O[p2]] : 1.f, p2 + 1 < k ? inv_s[O[p2 + 1]] : 1.f);
+    }
+    // X_O of ring row i (slot i mod kSlots, fill cycle i / kSlots); false if
+    // the wait for the row gave up
+    auto gather_outliers = [&](int64_t i) -> bool {
+      const int uu = static_cast<int>(i % R::kSlots);
+      if (!warp_wait_bounded(&full[uu], static_cast<uint32_t>((i / R::kSlots) & 1), abort_flag,
+                             DEVERR_TIMEOUT_PREP))
+        return false;
+      const uint8_t* slot = smem + static_cast<size_t>(uu) * R::kSlot;
+      uint32_t* xo_p = xo + (static_cast<int64_t>(blockIdx.x) + i * gridDim.x) * xo_pairs;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int pp = lane + 32 * q;
+        if (pp < xo_pairs) {
+          const float2 vv = __fmul2_rn(make_float2(pb_ring_f32(slot, po[2 * q]), pb_ring_f32(slot, po[2 * q + 1])),
+                                       pinv[q]);
+          xo_p[pp] = bf16_rn_bits(vv.x) | (bf16_rn_bits(vv.y) << 16);
+        }
+      }
+      for (int pp = lane + 64; pp < xo_pairs; pp += 32) {
+        const int o0 = 2 * pp;
+        const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : R::kZero;
+        const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : R::kZero;
+        const float y0 = __fmul_rn(pb_ring_f32(slot, a0), o0 < k ? inv_s[O[o0]] : 1.f);
+        const float y1 = __fmul_rn(pb_ring_f32(slot, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
+        xo_p[pp] = bf16_rn_bits(y0) | (bf16_rn_bits(y1) << 16);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[uu]);
+      return true;
+    };
     // failure-detection test hook: no copies at all, the consumers' waits run out
     const bool skip = (g_fault_mask & FAULT_PREP_SKIP_LOADS) != 0u;
     constexpr int G = R::kSlots / S;
@@ -97,10 +148,19 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
       int64_t issued = 0;
       int u = 0;
       uint32_t ph = 0;
+      bool failed = false;
       for (int64_t i = 0; i < nrows && !skip; ++i) {
-        if (i >= R::kSlots &&
-            !warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP))
-          break;
+        if (i >= R::kSlots) {
+          // the slot's previous row: its outliers, then the consumers' release
+          if (k > 0 && !gather_outliers(i - R::kSlots)) {
+            failed = true;
+            break;
+          }
+          if (!warp_wait_bounded(&empty[u], ph ^ 1u, abort_flag, DEVERR_TIMEOUT_PREP)) {
+            failed = true;
+            break;
+          }
+        }
         if (elect_one()) {
           mbar_arrive_expect_tx(&full[u], bytes);
           const int64_t r = blockIdx.x + i * gridDim.x;
@@ -115,6 +175,9 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
           ph ^= 1u;
         }
       }
+      // the outliers of the last rows in the ring
+      for (int64_t i = issued > R::kSlots ? issued - R::kSlots : 0; k > 0 && !failed && i < issued; ++i)
+        failed = !gather_outliers(i);
       if (lane == 0 && *abort_flag) {
         // do not leave bulk copies in flight into shared memory we give back
         const int64_t first = issued > R::kSlots ? issued - R::kSlots : 0;
@@ -232,21 +295,19 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
     go[e + 1] = gbase + o1;
     isv[e >> 1] = make_float2(i0, i1);
   }
-  // the outlier pair this thread gathers on every row (more pairs than
-  // threads only when k > 2 * ntg; those run through the loop below)
-  const int xo_row = k_pad >> 1;                            // bf16 pairs per row of X_O
-  uint32_t oo0 = R::kZero, oo1 = R::kZero;
-  float2 oinv = make_float2(1.f, 1.f);
-  if (t < xo_row) {
-    const int o0 = 2 * t;
-    if (o0 < k) {
-      oo0 = 2u * static_cast<uint32_t>(O[o0]);
-      oinv.x = inv_s[O[o0]];
-    }
-    if (o0 + 1 < k) {
-      oo1 = 2u * static_cast<uint32_t>(O[o0 + 1]);
-      oinv.y = inv_s[O[o0 + 1]];
-    }
+  // with several groups the group's warps gather the rows' outliers in turn:
+  // this lane's pairs p = lane, lane + 32 (further ones read O and inv_s again)
+  constexpr bool kConsumerXo = R::kSlots / S > 1;
+  const int xo_pairs = k_pad >> 1;
+  const int gwarp = t >> 5, gwarps = ntg >> 5;              // warp within the group, warps per group
+  uint32_t po[4];
+  float2 pinv[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int p2 = 2 * (lane + 32 * q);
+    po[2 * q] = gbase + (p2 < k ? 2u * static_cast<uint32_t>(O[p2]) : R::kZero);
+    po[2 * q + 1] = gbase + (p2 + 1 < k ? 2u * static_cast<uint32_t>(O[p2 + 1]) : R::kZero);
+    pinv[q] = make_float2(p2 < k ? inv_s[O[p2]] : 1.f, p2 + 1 < k ? inv_s[O[p2 + 1]] : 1.f);
   }
   const int64_t aq_row = static_cast<int64_t>(nblk) * 16;   // bytes per row of codes
   // this lane's block in row 0 of the codes and of the scale atoms
@@ -257,9 +318,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   const uint32_t bs = 8u * (static_cast<uint32_t>(m) & 3u);  // ... then bits
   uint32_t ph = 0;
   bool ok = true;
+  int xo_turn = 0;                                          // the group's warp that takes this row's outliers
 
-  oo0 += gbase;
-  oo1 += gbase;
 
   for (int64_t i0 = 0; i0 < nrows && ok; i0 += R::kSlots) {
 #pragma unroll
@@ -271,7 +331,6 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         break;
       }
       const uint8_t* ring = smem + j * R::kSlot;          // compile-time offset (+ gbase in go)
-      const uint8_t* slot = ring + gbase;
       const int r = static_cast<int>(blockIdx.x + (i0 + u) * gridDim.x);   // T < 2^31
       float2 v[16];
       float amax = 0.f;
@@ -323,19 +382,26 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         sfa_lane[static_cast<int64_t>(static_cast<uint32_t>(r) >> 7) * atom_row +
                  (((rl & 31u) << 4) | ((rl >> 5) << 2))] = static_cast<uint8_t>(code);
       }
-      if (t < xo_row) {
-        uint32_t* xo_p = xo + static_cast<int64_t>(r) * xo_row;
-        const float x0 = pb_ring_f32(ring, oo0);
-        const float x1 = pb_ring_f32(ring, oo1);
-        const float2 vv = __fmul2_rn(make_float2(x0, x1), oinv);
-        xo_p[t] = bf16_rn_bits(vv.x) | (bf16_rn_bits(vv.y) << 16);
-        for (int i2 = t + ntg; i2 < xo_row; i2 += ntg) {
-          const int o0 = 2 * i2;
-          const uint32_t a0 = o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : R::kZero;
-          const uint32_t a1 = o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : R::kZero;
-          const float y0 = __fmul_rn(pb_ring_f32(slot, a0), o0 < k ? inv_s[O[o0]] : 1.f);
-          const float y1 = __fmul_rn(pb_ring_f32(slot, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
-          xo_p[i2] = bf16_rn_bits(y0) | (bf16_rn_bits(y1) << 16);
+      const bool my_turn = xo_turn == gwarp;
+      if (++xo_turn == gwarps) xo_turn = 0;
+      if (kConsumerXo && k > 0 && my_turn) {
+        uint32_t* xo_p = xo + static_cast<int64_t>(r) * xo_pairs;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int pp = lane + 32 * q;
+          if (pp < xo_pairs) {
+            const float2 vv = __fmul2_rn(make_float2(pb_ring_f32(ring, po[2 * q]), pb_ring_f32(ring, po[2 * q + 1])),
+                                         pinv[q]);
+            xo_p[pp] = bf16_rn_bits(vv.x) | (bf16_rn_bits(vv.y) << 16);
+          }
+        }
+        for (int pp = lane + 64; pp < xo_pairs; pp += 32) {
+          const int o0 = 2 * pp;
+          const uint32_t a0 = gbase + (o0 < k ? 2u * static_cast<uint32_t>(O[o0]) : R::kZero);
+          const uint32_t a1 = gbase + (o0 + 1 < k ? 2u * static_cast<uint32_t>(O[o0 + 1]) : R::kZero);
+          const float y0 = __fmul_rn(pb_ring_f32(ring, a0), o0 < k ? inv_s[O[o0]] : 1.f);
+          const float y1 = __fmul_rn(pb_ring_f32(ring, a1), o0 + 1 < k ? inv_s[O[o0 + 1]] : 1.f);
+          xo_p[pp] = bf16_rn_bits(y0) | (bf16_rn_bits(y1) << 16);
         }
       }
       __syncwarp();

@@ -186,9 +186,10 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
                             nullptr, DEVERR_TIMEOUT_PREP);
       }
     } else {
-      // Rows go to the groups' slots in a fixed pattern (row i to slot i mod
-      // kSlots; group g owns slots g*S .. g*S + S - 1), and each group consumes
-      // its rows in order.  The producer refills whichever group's next slot is
+      // Rows go to the groups' slots in a fixed pattern (row i to group
+      // i mod G, which owns slots g*S .. g*S + S - 1 and takes its rows in
+      // turn -- groups' row counts differ by one at most), and each group
+      // consumes its rows in order.  The producer refills whichever group's next slot is
       // free, so one slow group does not hold back the others' refills.
       int gc[G], gj[G];                       // per group: ring cycle and slot of its next row
 #pragma unroll
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
         bool left = false, progress = false;
 #pragma unroll
         for (int q = 0; q < G; ++q) {
-          const int64_t i = static_cast<int64_t>(R::kSlots) * gc[q] + q * S + gj[q];
+          const int64_t i = (static_cast<int64_t>(gc[q]) * S + gj[q]) * G + q;
           if (i >= nrows) continue;
           left = true;
           const int u = q * S + gj[q];
@@ -321,17 +322,23 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
   int xo_turn = 0;                                          // the group's warp that takes this row's outliers
 
 
-  for (int64_t i0 = 0; i0 < nrows && ok; i0 += R::kSlots) {
+  // this group's rows: g, g + G, g + 2G, ... (CTA-local), in its slots g*S + j
+  constexpr int G = R::kSlots / S;
+  for (int64_t n0 = 0; ok; n0 += S) {
 #pragma unroll
     for (int j = 0; j < S; ++j) {
       const int u = g * S + j;
-      if (i0 + u >= nrows) break;
+      const int64_t i = (n0 + j) * G + g;
+      if (i >= nrows) {
+        ok = false;                         // no rows left (not an error)
+        break;
+      }
       if (!warp_wait_bounded(&full[u], ph, abort_flag, DEVERR_TIMEOUT_PREP)) {
         ok = false;
         break;
       }
       const uint8_t* ring = smem + j * R::kSlot;          // compile-time offset (+ gbase in go)
-      const int r = static_cast<int>(blockIdx.x + (i0 + u) * gridDim.x);   // T < 2^31
+      const int r = static_cast<int>(blockIdx.x + i * gridDim.x);   // T < 2^31
       float2 v[16];
       float amax = 0.f;
       if (enc) {

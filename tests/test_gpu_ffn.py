@@ -22,9 +22,13 @@ pytestmark = pytest.mark.gpu
 XS = synth.XSpec("student3", 0.3, 6, 8.0, 30.0)
 
 
-def test_gelu_every_bf16():
-    # all 65536 inputs, infinities and NaNs included (+inf -> +inf, -inf and NaN -> NaN)
-    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+@pytest.mark.parametrize("shift", [0, 1])
+def test_gelu_every_bf16(shift):
+    # all 65536 inputs, infinities and NaNs included (+inf -> +inf, -inf and NaN -> NaN);
+    # the kernel works on bf16 pairs, so each input is checked in the low half
+    # (shift 0) and in the high half (shift 1) of its pair -- the same function
+    # the fused GEMM epilogue evaluates
+    bits = np.roll(np.arange(65536, dtype=np.uint32).astype(np.uint16), shift)
     Y = torch.from_numpy(bits.view(np.int16).reshape(-1, 64)).cuda().view(torch.bfloat16)
     H = ffn.gelu_bf16(Y)
     torch.cuda.synchronize()

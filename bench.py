@@ -357,16 +357,15 @@ class LayerRun:
         w4, L, pw = self.w4, self.L, self.pw
         if ev is not None:
             ev[0].record()
-        w4.calib_observe(self.X, pw.act_scale, reset=True)
-        w4.calib_observe(self.W, pw.w_scale, reset=True)
+        w4.calib_observe_layer(self.X, self.W, pw.act_scale, pw.w_scale, reset=True)
         if ev is not None:
             ev[1].record()
         w4.calib_finalize(pw.act_scale, pw.w_scale, L.alpha, L.k, pw.s, pw.inv_s, pw.score,
                           pw.O if L.k else None, pw.jmap if L.k < L.d_in else None)
         w4.pack_weight(self.W, pw)
-        # colabsmax x2, finalize x2, pack: one prep launch (32x1) or tile + bf16 kernels (32x32)
+        # colabsmax (X and W), finalize x2, pack: one prep launch (32x1) or tile + bf16 kernels (32x32)
         pack = 1 if L.layout in (0, 2) else (1 if self.d.kj else 0) + (1 if L.k else 0)
-        return 4 + pack
+        return 3 + pack
 
     def online(self, ev=None):
         w4 = self.w4

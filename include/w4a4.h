@@ -109,6 +109,18 @@ w4a4_status w4a4_get_dims(int64_t d_in, int64_t d_out, int64_t k, w4a4_dims* out
 w4a4_status w4a4_calib_observe(const void* A, int64_t rows, int64_t cols, int64_t lda,
                                float* absmax, int reset, void* stream);
 
+/* One layer's magnitudes from one batch in one launch: the column absmax of
+ * X [T, d_in] (row stride ldx) into act_absmax and of W [d_out, d_in] (row
+ * stride ldw) into w_absmax, both float32 [d_in] -- the values of
+ * w4a4_calib_observe on X and on W (reset applies to both).  T or d_out may
+ * be 0.  Further activation batches go through w4a4_calib_observe with
+ * reset = 0.  Errors: INVALID_ARG for null or negative arguments, strides
+ * below d_in or act_absmax == w_absmax; UNSUPPORTED_SHAPE unless d_in, ldx
+ * and ldw are multiples of 8 and X and W are 16-byte aligned. */
+w4a4_status w4a4_calib_observe_layer(const void* X, int64_t T, int64_t ldx, const void* W,
+                                     int64_t d_out, int64_t ldw, int64_t d_in, float* act_absmax,
+                                     float* w_absmax, int reset, void* stream);
+
 /* From act_scale and w_scale (float32 [d_in]) compute, on the device:
  *   s[j]     = fl32( max(a,1e-5)^alpha / max(w,1e-5)^(1-alpha) )  in float64
  *   inv_s[j] = fl32( 1 / s[j] )

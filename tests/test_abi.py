@@ -166,6 +166,18 @@ def test_calib_validation():
     assert w4._calib_observe(0x1000, 4, 12, 12, 0x1000, 1, None) == w4.ERR_UNSUPPORTED_SHAPE
     assert w4._calib_observe(None, 4, 8, 8, 0x1000, 1, None) == w4.ERR_INVALID_ARG
     f = 0x1000
+    # the one-launch layer form: X [T, d_in] and W [d_out, d_in]
+    lay = w4._calib_observe_layer
+    assert lay(f, 4, 8, f, 4, 8, 8, f, f, 1, None) == w4.ERR_INVALID_ARG          # outputs alias
+    assert lay(f, 4, 8, f, 4, 8, 8, None, f + 64, 1, None) == w4.ERR_INVALID_ARG
+    assert lay(f, 4, 4, f, 4, 8, 8, f, f + 64, 1, None) == w4.ERR_INVALID_ARG     # ldx < d_in
+    assert lay(f, 4, 8, f, 4, 4, 8, f, f + 64, 1, None) == w4.ERR_INVALID_ARG     # ldw < d_in
+    assert lay(None, 4, 8, f, 4, 8, 8, f, f + 64, 1, None) == w4.ERR_INVALID_ARG  # X missing
+    assert lay(f, 4, 8, None, 4, 8, 8, f, f + 64, 1, None) == w4.ERR_INVALID_ARG  # W missing
+    assert lay(f, -1, 8, f, 4, 8, 8, f, f + 64, 1, None) == w4.ERR_INVALID_ARG
+    assert lay(f, 4, 12, f, 4, 12, 12, f, f + 64, 1, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert lay(f + 8, 4, 8, f, 4, 8, 8, f, f + 64, 1, None) == w4.ERR_UNSUPPORTED_SHAPE
+    assert lay(None, 0, 8, None, 0, 8, 8, f, f + 64, 0, None) == w4.OK            # nothing to do
     assert w4._calib_finalize(f, f, 64, 0.0, 4, f, f, f, f, f, None) == w4.ERR_INVALID_ARG   # alpha
     assert w4._calib_finalize(f, f, 64, 1.0, 4, f, f, f, f, f, None) == w4.ERR_INVALID_ARG
     assert w4._calib_finalize(f, f, 64, 0.5, 65, f, f, f, f, f, None) == w4.ERR_INVALID_ARG  # k > d_in

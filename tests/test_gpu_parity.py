@@ -163,6 +163,30 @@ def test_calibration_multi_batch_running_max():
     np.testing.assert_array_equal(pw.act_scale.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("T,d_out,d_in", [(200, 368, 136), (0, 96, 64), (300, 0, 64),
+                                           (57, 1000 - 8, 5120), (4096, 32, 8)])
+def test_calibration_layer_call(T, d_out, d_in):
+    """X and W in one launch: the values of two single-matrix calls, and of the
+    column absmax by its definition; reset = 0 keeps the running maximum."""
+    g = torch.Generator().manual_seed(T * 7 + d_out)
+    X = (torch.randn(T, d_in, generator=g) * 3).to(torch.bfloat16).cuda()
+    W = (torch.randn(d_out, d_in, generator=g) * 0.05).to(torch.bfloat16).cuda()
+    f = lambda: torch.full((d_in,), 7.0, device="cuda")
+    a1, w1, a2, w2 = f(), f(), f(), f()
+    w4.calib_observe_layer(X, W, a1, w1, reset=True)
+    w4.calib_observe(X, a2, reset=True)
+    w4.calib_observe(W, w2, reset=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, a2) and torch.equal(w1, w2)
+    np.testing.assert_array_equal(a1.cpu().numpy(), orc.col_absmax(gu.to_np_f32(X)))
+    np.testing.assert_array_equal(w1.cpu().numpy(), orc.col_absmax(gu.to_np_f32(W)))
+    # running maximum: a second call without reset on half-size inputs changes nothing
+    w4.calib_observe_layer((X.float() * 0.5).to(torch.bfloat16), (W.float() * 0.5).to(torch.bfloat16),
+                           a1, w1, reset=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, a2) and torch.equal(w1, w2)
+
+
 def test_topk_ties_go_to_lower_index():
     d_in, k = 64, 5
     act = torch.ones(d_in, device="cuda")

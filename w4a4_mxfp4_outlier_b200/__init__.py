@@ -60,6 +60,8 @@ _status_string = _sig("w4a4_status_string", ctypes.c_char_p, _st)
 _num_sms = _sig("w4a4_num_sms", ctypes.c_int)
 _get_dims = _sig("w4a4_get_dims", _st, _i64, _i64, _i64, ctypes.POINTER(Dims))
 _calib_observe = _sig("w4a4_calib_observe", _st, _vp, _i64, _i64, _i64, _vp, ctypes.c_int, _vp)
+_calib_observe_layer = _sig("w4a4_calib_observe_layer", _st, _vp, _i64, _i64, _vp, _i64, _i64, _i64,
+                            _vp, _vp, ctypes.c_int, _vp)
 _calib_finalize = _sig("w4a4_calib_finalize", _st, _vp, _vp, _i64, ctypes.c_double, _i64,
                        _vp, _vp, _vp, _vp, _vp, _vp)
 _weight_sizes = _sig("w4a4_weight_sizes", _st, _i64, _i64, _i64, ctypes.POINTER(WeightBytes))
@@ -100,7 +102,8 @@ FAULT_PREP_SKIP_LOADS = 1           # W4A4_FAULT_PREP_SKIP_LOADS
 
 EXPORTED = [
     "w4a4_abi_version", "w4a4_status_string", "w4a4_num_sms", "w4a4_get_dims",
-    "w4a4_calib_observe", "w4a4_calib_finalize", "w4a4_weight_sizes", "w4a4_pack_weight",
+    "w4a4_calib_observe", "w4a4_calib_observe_layer", "w4a4_calib_finalize", "w4a4_weight_sizes",
+    "w4a4_pack_weight",
     "w4a4_workspace_size", "w4a4_prep_act", "w4a4_gemm_dual", "w4a4_linear",
     "w4a4_linear_host", "w4a4_linear_noalloc", "w4a4_last_error",
     "w4a4_packed_image_size", "w4a4_packed_save", "w4a4_packed_image_info", "w4a4_packed_load",
@@ -186,6 +189,19 @@ def calib_observe(A: torch.Tensor, absmax: torch.Tensor, reset: bool, stream=Non
                           _stream(stream)), "calib_observe")
 
 
+def calib_observe_layer(X: torch.Tensor, W: torch.Tensor, act_scale: torch.Tensor,
+                        w_scale: torch.Tensor, reset: bool, stream=None):
+    """Column absmax of X into act_scale and of W into w_scale, one launch."""
+    _rows_bf16(X, "calib_observe_layer", act_scale.device)
+    _rows_bf16(W, "calib_observe_layer", act_scale.device)
+    if X.shape[1] != W.shape[1]:
+        raise W4A4Error(ERR_INVALID_ARG, f"calib_observe_layer: X has {X.shape[1]} columns, "
+                        f"W {W.shape[1]}")
+    _check(_calib_observe_layer(_ptr(X), X.shape[0], X.stride(0), _ptr(W), W.shape[0], W.stride(0),
+                                X.shape[1], _ptr(act_scale), _ptr(w_scale), int(reset),
+                                _stream(stream)), "calib_observe_layer")
+
+
 def calib_finalize(act_scale, w_scale, alpha: float, k: int, s, inv_s, score, O, jmap, stream=None):
     _check(_calib_finalize(_ptr(act_scale), _ptr(w_scale), act_scale.numel(), float(alpha), k,
                            _ptr(s), _ptr(inv_s), _ptr(score), _ptr(O), _ptr(jmap),
@@ -247,15 +263,16 @@ def pack_weight(W: torch.Tensor, pw: PackedWeight, stream=None):
 
 def calibrate(X_batches, W: torch.Tensor, alpha: float, k: int,
               layout: int = SF_32x1_KMAJOR, stream=None) -> PackedWeight:
-    """calib_observe over the activation batches and W, calib_finalize, then
-    pack_weight: the offline half of the method, all on the device."""
+    """Column absmax of the first activation batch and W (one launch), of the
+    further batches (running maximum), calib_finalize, then pack_weight: the
+    offline half of the method, all on the device."""
     if isinstance(X_batches, torch.Tensor):
         X_batches = [X_batches]
     d_out, d_in = W.shape
     pw = alloc_packed(d_in, d_out, k, layout, W.device)
-    for i, Xb in enumerate(X_batches):
-        calib_observe(Xb, pw.act_scale, reset=(i == 0), stream=stream)
-    calib_observe(W, pw.w_scale, reset=True, stream=stream)
+    calib_observe_layer(X_batches[0], W, pw.act_scale, pw.w_scale, reset=True, stream=stream)
+    for Xb in X_batches[1:]:
+        calib_observe(Xb, pw.act_scale, reset=False, stream=stream)
     calib_finalize(pw.act_scale, pw.w_scale, alpha, k, pw.s, pw.inv_s, pw.score,
                    pw.O if k else None, pw.jmap if k < d_in else None, stream=stream)
     pack_weight(W, pw, stream=stream)

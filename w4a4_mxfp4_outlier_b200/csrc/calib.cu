@@ -9,23 +9,39 @@
 namespace w4a4 {
 
 // ---------------------------------------------------------------------------
-// Column absmax.  Block = 32 x 8 threads; threadIdx.x owns 8 consecutive
-// columns (one 16-byte load per row), threadIdx.y and blockIdx.y stride over
-// rows.  Magnitudes are compared as bf16 bit patterns with the sign cleared
-// (for non-NaN values the integer order is the magnitude order), packed two
-// per 32-bit word.  The block result goes to global memory with an integer
-// atomicMax on the float32 bits, which orders non-negative floats correctly.
+// Column absmax of one or two matrices with the same columns (a layer's X
+// and W share d_in) in one launch.  Block = 32 x 8 threads; threadIdx.x owns
+// 8 consecutive columns (one 16-byte load per row), threadIdx.y and the
+// block row stride over rows; block rows 0 .. p0.gy-1 reduce p0, the others
+// p1.  Magnitudes are compared as bf16 bit patterns with the sign cleared
+// (for non-NaN values the integer order is the magnitude order; NaN patterns
+// lie above +inf, so a NaN makes the column NaN), packed two per 32-bit
+// word.  The block result goes to global memory with an integer atomicMax
+// on the float32 bits, which orders non-negative floats correctly.
 // HBM-bound: 2 bytes read per element.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) colabsmax_kernel(const uint16_t* __restrict__ A,
-                                                        int64_t rows, int64_t cols, int64_t lda,
-                                                        uint32_t* __restrict__ out_bits) {
+struct AbsmaxPart {
+  const uint16_t* A;
+  int64_t rows, lda;
+  uint32_t* out;     // float32 bits [cols]
+  int gy;            // block rows given to this matrix
+};
+
+__global__ void __launch_bounds__(256) colabsmax_kernel(const AbsmaxPart p0, const AbsmaxPart p1,
+                                                        int64_t cols) {
   __shared__ uint32_t red[8][32][4];
+  const bool second = static_cast<int>(blockIdx.y) >= p0.gy;
+  const uint16_t* A = second ? p1.A : p0.A;
+  const int64_t rows = second ? p1.rows : p0.rows;
+  const int64_t lda = second ? p1.lda : p0.lda;
+  const int gy = second ? p1.gy : p0.gy;
+  const int by = second ? static_cast<int>(blockIdx.y) - p0.gy : static_cast<int>(blockIdx.y);
   const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.x) * 8;
+  constexpr uint32_t kMag = 0x7FFF7FFFu;
   uint32_t m[4] = {0u, 0u, 0u, 0u};
   if (col0 < cols) {
-    const int64_t rstep = static_cast<int64_t>(gridDim.y) * 8;
-    int64_t r = static_cast<int64_t>(blockIdx.y) * 8 + threadIdx.y;
+    const int64_t rstep = static_cast<int64_t>(gy) * 8;
+    int64_t r = static_cast<int64_t>(by) * 8 + threadIdx.y;
     const uint16_t* p = A + col0;
     // eight rows in flight per iteration, folded pairwise (measured against
     // four: 5.98 -> 6.61 TB/s on a 57600 x 5120 X)
@@ -38,29 +54,25 @@ __global__ void __launch_bounds__(256) colabsmax_kernel(const uint16_t* __restri
       uint4 v1 = __ldcs(reinterpret_cast<const uint4*>(p + (r + rstep) * lda));
       uint4 v2 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 2 * rstep) * lda));
       uint4 v3 = __ldcs(reinterpret_cast<const uint4*>(p + (r + 3 * rstep) * lda));
-      v0.x = __vmaxu2(v0.x & 0x7FFF7FFFu, u0.x & 0x7FFF7FFFu); v0.y = __vmaxu2(v0.y & 0x7FFF7FFFu, u0.y & 0x7FFF7FFFu);
-      v0.z = __vmaxu2(v0.z & 0x7FFF7FFFu, u0.z & 0x7FFF7FFFu); v0.w = __vmaxu2(v0.w & 0x7FFF7FFFu, u0.w & 0x7FFF7FFFu);
-      v1.x = __vmaxu2(v1.x & 0x7FFF7FFFu, u1.x & 0x7FFF7FFFu); v1.y = __vmaxu2(v1.y & 0x7FFF7FFFu, u1.y & 0x7FFF7FFFu);
-      v1.z = __vmaxu2(v1.z & 0x7FFF7FFFu, u1.z & 0x7FFF7FFFu); v1.w = __vmaxu2(v1.w & 0x7FFF7FFFu, u1.w & 0x7FFF7FFFu);
-      v2.x = __vmaxu2(v2.x & 0x7FFF7FFFu, u2.x & 0x7FFF7FFFu); v2.y = __vmaxu2(v2.y & 0x7FFF7FFFu, u2.y & 0x7FFF7FFFu);
-      v2.z = __vmaxu2(v2.z & 0x7FFF7FFFu, u2.z & 0x7FFF7FFFu); v2.w = __vmaxu2(v2.w & 0x7FFF7FFFu, u2.w & 0x7FFF7FFFu);
-      v3.x = __vmaxu2(v3.x & 0x7FFF7FFFu, u3.x & 0x7FFF7FFFu); v3.y = __vmaxu2(v3.y & 0x7FFF7FFFu, u3.y & 0x7FFF7FFFu);
-      v3.z = __vmaxu2(v3.z & 0x7FFF7FFFu, u3.z & 0x7FFF7FFFu); v3.w = __vmaxu2(v3.w & 0x7FFF7FFFu, u3.w & 0x7FFF7FFFu);
-      m[0] = __vmaxu2(m[0], __vmaxu2(__vmaxu2(v0.x & 0x7FFF7FFFu, v1.x & 0x7FFF7FFFu),
-                                     __vmaxu2(v2.x & 0x7FFF7FFFu, v3.x & 0x7FFF7FFFu)));
-      m[1] = __vmaxu2(m[1], __vmaxu2(__vmaxu2(v0.y & 0x7FFF7FFFu, v1.y & 0x7FFF7FFFu),
-                                     __vmaxu2(v2.y & 0x7FFF7FFFu, v3.y & 0x7FFF7FFFu)));
-      m[2] = __vmaxu2(m[2], __vmaxu2(__vmaxu2(v0.z & 0x7FFF7FFFu, v1.z & 0x7FFF7FFFu),
-                                     __vmaxu2(v2.z & 0x7FFF7FFFu, v3.z & 0x7FFF7FFFu)));
-      m[3] = __vmaxu2(m[3], __vmaxu2(__vmaxu2(v0.w & 0x7FFF7FFFu, v1.w & 0x7FFF7FFFu),
-                                     __vmaxu2(v2.w & 0x7FFF7FFFu, v3.w & 0x7FFF7FFFu)));
+      v0.x = __vmaxu2(v0.x & kMag, u0.x & kMag); v0.y = __vmaxu2(v0.y & kMag, u0.y & kMag);
+      v0.z = __vmaxu2(v0.z & kMag, u0.z & kMag); v0.w = __vmaxu2(v0.w & kMag, u0.w & kMag);
+      v1.x = __vmaxu2(v1.x & kMag, u1.x & kMag); v1.y = __vmaxu2(v1.y & kMag, u1.y & kMag);
+      v1.z = __vmaxu2(v1.z & kMag, u1.z & kMag); v1.w = __vmaxu2(v1.w & kMag, u1.w & kMag);
+      v2.x = __vmaxu2(v2.x & kMag, u2.x & kMag); v2.y = __vmaxu2(v2.y & kMag, u2.y & kMag);
+      v2.z = __vmaxu2(v2.z & kMag, u2.z & kMag); v2.w = __vmaxu2(v2.w & kMag, u2.w & kMag);
+      v3.x = __vmaxu2(v3.x & kMag, u3.x & kMag); v3.y = __vmaxu2(v3.y & kMag, u3.y & kMag);
+      v3.z = __vmaxu2(v3.z & kMag, u3.z & kMag); v3.w = __vmaxu2(v3.w & kMag, u3.w & kMag);
+      m[0] = __vmaxu2(m[0], __vmaxu2(__vmaxu2(v0.x, v1.x), __vmaxu2(v2.x, v3.x)));
+      m[1] = __vmaxu2(m[1], __vmaxu2(__vmaxu2(v0.y, v1.y), __vmaxu2(v2.y, v3.y)));
+      m[2] = __vmaxu2(m[2], __vmaxu2(__vmaxu2(v0.z, v1.z), __vmaxu2(v2.z, v3.z)));
+      m[3] = __vmaxu2(m[3], __vmaxu2(__vmaxu2(v0.w, v1.w), __vmaxu2(v2.w, v3.w)));
     }
     for (; r < rows; r += rstep) {
       uint4 v = __ldcs(reinterpret_cast<const uint4*>(p + r * lda));
-      m[0] = __vmaxu2(m[0], v.x & 0x7FFF7FFFu);
-      m[1] = __vmaxu2(m[1], v.y & 0x7FFF7FFFu);
-      m[2] = __vmaxu2(m[2], v.z & 0x7FFF7FFFu);
-      m[3] = __vmaxu2(m[3], v.w & 0x7FFF7FFFu);
+      m[0] = __vmaxu2(m[0], v.x & kMag);
+      m[1] = __vmaxu2(m[1], v.y & kMag);
+      m[2] = __vmaxu2(m[2], v.z & kMag);
+      m[3] = __vmaxu2(m[3], v.w & kMag);
     }
   }
 #pragma unroll
@@ -71,33 +83,70 @@ __global__ void __launch_bounds__(256) colabsmax_kernel(const uint16_t* __restri
     for (int y = 1; y < 8; ++y)
 #pragma unroll
       for (int i = 0; i < 4; ++i) m[i] = __vmaxu2(m[i], red[y][threadIdx.x][i]);
+    uint32_t* out = second ? p1.out : p0.out;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       // low half = column col0 + 2i, high half = col0 + 2i + 1; bf16 -> f32 bits
-      atomicMax(out_bits + col0 + 2 * i, (m[i] & 0xFFFFu) << 16);
-      atomicMax(out_bits + col0 + 2 * i + 1, m[i] & 0xFFFF0000u);
+      atomicMax(out + col0 + 2 * i, (m[i] & 0xFFFFu) << 16);
+      atomicMax(out + col0 + 2 * i + 1, m[i] & 0xFFFF0000u);
     }
   }
 }
 
-cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
-                             int reset, cudaStream_t stream) {
+// Resident blocks of colabsmax_kernel per SM (cached per device).
+static int colabsmax_blocks_per_sm() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colabsmax_kernel, 256, 0) != cudaSuccess ||
+        n <= 0)
+      n = 4;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// One launch over A0 (rows0 rows) and, if rows1 > 0, A1, both `cols` wide.
+// The grid is one wave of resident blocks (a second, partial wave left a
+// tail: 0.1345 -> 0.1262 ms for X and W of the 5120-column layer at
+// T = 57600 with both in one launch), its block rows split between the two
+// matrices in proportion to their rows, at least 4 rows per thread.
+cudaError_t launch_colabsmax2(const void* A0, int64_t rows0, int64_t lda0, float* out0,
+                              const void* A1, int64_t rows1, int64_t lda1, float* out1,
+                              int64_t cols, int reset, cudaStream_t stream) {
   if (reset) {
-    cudaError_t e = cudaMemsetAsync(absmax, 0, static_cast<size_t>(cols) * sizeof(float), stream);
+    cudaError_t e = cudaMemsetAsync(out0, 0, static_cast<size_t>(cols) * sizeof(float), stream);
+    if (e == cudaSuccess && out1 != nullptr)
+      e = cudaMemsetAsync(out1, 0, static_cast<size_t>(cols) * sizeof(float), stream);
     if (e != cudaSuccess) return e;
   }
-  if (rows == 0 || cols == 0) return cudaSuccess;
-  const int sms = device_num_sms();
+  if (cols == 0 || rows0 + rows1 == 0) return cudaSuccess;
+  const int64_t sms = device_num_sms() > 0 ? device_num_sms() : 148;
   const int64_t gx = (cols + 255) / 256;
-  int64_t want = (static_cast<int64_t>(sms) * 8 + gx - 1) / gx;      // ~8 blocks per SM
-  int64_t maxy = (rows + 31) / 32;                                    // >= 4 rows per thread
-  int64_t gy = want < maxy ? want : maxy;
-  if (gy < 1) gy = 1;
-  if (gy > 65535) gy = 65535;
-  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-  colabsmax_kernel<<<grid, dim3(32, 8), 0, stream>>>(static_cast<const uint16_t*>(A), rows, cols,
-                                                     lda, reinterpret_cast<uint32_t*>(absmax));
+  int64_t total = sms * colabsmax_blocks_per_sm() / gx;
+  if (total < 2) total = 2;
+  auto cap = [](int64_t gy, int64_t rows) -> int64_t {
+    if (rows == 0) return 0;
+    const int64_t maxy = (rows + 31) / 32;               // >= 4 rows per thread
+    if (gy > maxy) gy = maxy;
+    return gy < 1 ? 1 : gy;
+  };
+  const int64_t gy0 = cap((total * rows0 + (rows0 + rows1) / 2) / (rows0 + rows1), rows0);
+  const int64_t gy1 = cap(total - gy0, rows1);
+  AbsmaxPart p0{static_cast<const uint16_t*>(A0), rows0, lda0, reinterpret_cast<uint32_t*>(out0),
+                static_cast<int>(gy0)};
+  AbsmaxPart p1{static_cast<const uint16_t*>(A1), rows1, lda1, reinterpret_cast<uint32_t*>(out1),
+                static_cast<int>(gy1)};
+  colabsmax_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy0 + gy1)), dim3(32, 8),
+                     0, stream>>>(p0, p1, cols);
   return cudaGetLastError();
+}
+
+cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
+                             int reset, cudaStream_t stream) {
+  return launch_colabsmax2(A, rows, lda, absmax, nullptr, 0, lda, nullptr, cols, reset, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -172,6 +172,19 @@ w4a4_status w4a4_calib_observe(const void* A, int64_t rows, int64_t cols, int64_
                                     static_cast<cudaStream_t>(stream)));
 }
 
+w4a4_status w4a4_calib_observe_layer(const void* X, int64_t T, int64_t ldx, const void* W,
+                                     int64_t d_out, int64_t ldw, int64_t d_in, float* act_absmax,
+                                     float* w_absmax, int reset, void* stream) {
+  if (act_absmax == nullptr || w_absmax == nullptr || act_absmax == w_absmax || T < 0 ||
+      d_out < 0 || d_in <= 0 || ldx < d_in || ldw < d_in)
+    return W4A4_ERR_INVALID_ARG;
+  if ((T > 0 && X == nullptr) || (d_out > 0 && W == nullptr)) return W4A4_ERR_INVALID_ARG;
+  if (d_in % 8 != 0 || ldx % 8 != 0 || ldw % 8 != 0 || (X && !aligned16(X)) || (W && !aligned16(W)))
+    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_colabsmax2(X, T, ldx, act_absmax, W, d_out, ldw, w_absmax, d_in, reset,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 w4a4_status w4a4_calib_finalize(const float* act_scale, const float* w_scale, int64_t d_in,
                                 double alpha, int64_t k, float* s, float* inv_s, float* score,
                                 int32_t* O, int32_t* jmap, void* stream) {

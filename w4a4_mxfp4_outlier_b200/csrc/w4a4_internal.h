@@ -47,6 +47,10 @@ int device_num_sms();
 
 cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
                              int reset, cudaStream_t stream);
+// both matrices in one launch (A1 may have 0 rows; out1 is then unused)
+cudaError_t launch_colabsmax2(const void* A0, int64_t rows0, int64_t lda0, float* out0,
+                              const void* A1, int64_t rows1, int64_t lda1, float* out1,
+                              int64_t cols, int reset, cudaStream_t stream);
 cudaError_t launch_finalize(const float* act, const float* wsc, int d_in, double alpha, int k,
                             float* s, float* inv_s, float* score, int32_t* O, int32_t* jmap,
                             cudaStream_t stream);

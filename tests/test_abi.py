@@ -271,3 +271,21 @@ def test_fault_hook_validates_before_touching_the_device():
     assert w4._test_fault(2, 0) == w4.ERR_INVALID_ARG
     assert w4._test_fault(1, 3_000_000_000) == w4.ERR_INVALID_ARG
     assert "inf or NaN" in w4.status_string(w4.ERR_NONFINITE_CALIB)
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package without libw4a4.so refuses to import (no
+    fallback path of any kind)."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.dirname(w4.__file__)
+    dst = tmp_path / "w4a4_mxfp4_outlier_b200"
+    dst.mkdir()
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            shutil.copy(os.path.join(pkg, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import w4a4_mxfp4_outlier_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libw4a4.so is not built" in r.stderr

@@ -4,8 +4,8 @@ Argument marshalling only: every step of the computation runs in the CUDA
 kernels of ``libw4a4.so``; torch supplies device memory and streams.  The
 functions carry the names of the C entry points in ``include/w4a4.h``
 without the ``w4a4_`` prefix.  Importing this module fails loudly when the
-shared library is missing (build it with ``python -m
-w4a4_mxfp4_outlier_b200.build``); there is no fallback of any kind.
+shared library is missing (build it with ``python
+w4a4_mxfp4_outlier_b200/build.py``); there is no fallback of any kind.
 """
 from __future__ import annotations
 

@@ -30,6 +30,8 @@ struct AbsmaxPart {
 __global__ void __launch_bounds__(256) colabsmax_kernel(const AbsmaxPart p0, const AbsmaxPart p1,
                                                         int64_t cols) {
   __shared__ uint32_t red[8][32][4];
+  pdl_wait();
+  pdl_launch_dependents();
   const bool second = static_cast<int>(blockIdx.y) >= p0.gy;
   const uint16_t* A = second ? p1.A : p0.A;
   const int64_t rows = second ? p1.rows : p0.rows;
@@ -139,9 +141,8 @@ cudaError_t launch_colabsmax2(const void* A0, int64_t rows0, int64_t lda0, float
                 static_cast<int>(gy0)};
   AbsmaxPart p1{static_cast<const uint16_t*>(A1), rows1, lda1, reinterpret_cast<uint32_t*>(out1),
                 static_cast<int>(gy1)};
-  colabsmax_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy0 + gy1)), dim3(32, 8),
-                     0, stream>>>(p0, p1, cols);
-  return cudaGetLastError();
+  return launch_pdl(colabsmax_kernel, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy0 + gy1)),
+                    dim3(32, 8), 0, stream, p0, p1, cols);
 }
 
 cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
@@ -155,6 +156,8 @@ cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t 
 __global__ void finalize_scales_kernel(const float* __restrict__ act, const float* __restrict__ wsc,
                                        int d_in, double alpha, float* __restrict__ s,
                                        float* __restrict__ inv_s, float* __restrict__ score) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d_in) return;
   // s is defined for finite magnitudes only: an infinite or NaN one (from
@@ -193,6 +196,8 @@ __global__ void __launch_bounds__(kFinalizeThreads)
   __shared__ uint32_t warp_cnt[kFinalizeThreads / 32];
   __shared__ uint64_t sel_prefix;
   __shared__ uint32_t sel_remaining;
+  pdl_wait();
+  pdl_launch_dependents();
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int per = (d_in + kFinalizeThreads - 1) / kFinalizeThreads;
@@ -302,11 +307,11 @@ cudaError_t launch_finalize(const float* act, const float* wsc, int d_in, double
                             float* s, float* inv_s, float* score, int32_t* O, int32_t* jmap,
                             cudaStream_t stream) {
   const int nb = (d_in + 255) / 256;
-  finalize_scales_kernel<<<nb, 256, 0, stream>>>(act, wsc, d_in, alpha, s, inv_s, score);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(finalize_scales_kernel, dim3(nb), dim3(256), 0, stream, act, wsc, d_in,
+                             alpha, s, inv_s, score);
   if (e != cudaSuccess) return e;
-  finalize_select_kernel<<<1, kFinalizeThreads, 0, stream>>>(score, d_in, k, O, jmap);
-  return cudaGetLastError();
+  return launch_pdl(finalize_select_kernel, dim3(1), dim3(kFinalizeThreads), 0, stream, score, d_in, k,
+                    O, jmap);
 }
 
 }  // namespace w4a4

@@ -256,6 +256,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();                  // barrier and tensor-memory setup overlap the previous kernel
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ============================ TMA producer ============================
@@ -577,6 +579,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync_all();          // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();                  // barrier and tensor-memory setup overlap the previous kernel
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ============================ TMA producer (both CTAs) ================
@@ -1155,13 +1159,13 @@ cudaError_t run_gemm(const GemmPlan& p, cudaStream_t stream) {
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1 + static_cast<unsigned>(pdl_attrs(&attr[1]));
     if (p.act)
       return cudaLaunchKernelEx(&cfg, gemm_dual_pair_kernel<true, 256>, p.tm_a, p.tm_b, p.tm_ao,
                                 p.tm_bo, p.tm_sfa, p.tm_sfb, p.tm_y, p.a);
@@ -1172,12 +1176,10 @@ cudaError_t run_gemm(const GemmPlan& p, cudaStream_t stream) {
                               p.tm_bo, p.tm_sfa, p.tm_sfb, p.tm_y, p.a);
   }
   if (p.act)
-    gemm_dual_kernel<true><<<p.grid, GEMM_THREADS, p.smem, stream>>>(p.tm_a, p.tm_b, p.tm_ao,
-                                                                      p.tm_bo, p.a);
-  else
-    gemm_dual_kernel<false><<<p.grid, GEMM_THREADS, p.smem, stream>>>(p.tm_a, p.tm_b, p.tm_ao,
-                                                                       p.tm_bo, p.a);
-  return cudaGetLastError();
+    return launch_pdl(gemm_dual_kernel<true>, dim3(p.grid), dim3(GEMM_THREADS), p.smem, stream, p.tm_a,
+                      p.tm_b, p.tm_ao, p.tm_bo, p.a);
+  return launch_pdl(gemm_dual_kernel<false>, dim3(p.grid), dim3(GEMM_THREADS), p.smem, stream, p.tm_a,
+                    p.tm_b, p.tm_ao, p.tm_bo, p.a);
 }
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* sfa, const void* xo, int64_t T,

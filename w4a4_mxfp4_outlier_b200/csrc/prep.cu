@@ -80,6 +80,8 @@ __global__ void __maxnreg__(PrepCfg<CH>::kMaxRegs) prep_kernel(const uint16_t* _
     *reinterpret_cast<uint4*>(smem + static_cast<size_t>(u) * kPrepStage + kPrepZero) =
         make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
+  pdl_wait();                  // the shared-memory setup above overlaps the previous kernel
+  pdl_launch_dependents();
 
   const int64_t nrows = T > blockIdx.x ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
@@ -286,12 +288,11 @@ static cudaError_t launch_prep_ch(const PrepPlan& p, int grid, const void* X, in
   cudaError_t e = cudaFuncSetAttribute(prep_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kPrepSmem));
   if (e != cudaSuccess) return e;
-  prep_kernel<CH><<<grid, p.nt + 32, kPrepSmem, stream>>>(
-      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
-      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
-      static_cast<int>(g.kj_pad / 8), static_cast<int>(g.nblk), aq, sfa,
-      static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
-  return cudaGetLastError();
+  return launch_pdl(prep_kernel<CH>, dim3(grid), dim3(p.nt + 32), kPrepSmem, stream,
+                    static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
+                    static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
+                    static_cast<int>(g.kj_pad / 8), static_cast<int>(g.nblk), aq, sfa,
+                    static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
 }
 
 cudaError_t launch_prep(const void* X, int64_t T, int64_t ldx, const float* inv_s,

@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kPbMaxThreads, 1)
     *reinterpret_cast<uint4*>(smem + static_cast<size_t>(u) * R::kSlot + R::kZero) =
         make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
+  pdl_wait();                  // the shared-memory setup above overlaps the previous kernel
+  pdl_launch_dependents();
 
   const int64_t nrows = T > blockIdx.x ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
@@ -450,11 +452,11 @@ static cudaError_t launch_prep_block_s(const PrepBlockPlan& p, const void* X, in
   if (e != cudaSuccess) return e;
   const int sms = device_num_sms();
   const int grid = static_cast<int>(T < sms ? T : sms);
-  prep_block_kernel<S, R><<<grid, p.groups * p.ntg + 32, R::kSmem, stream>>>(
-      static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
-      static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
-      static_cast<int>(g.nblk), p.ntg, aq, sfa, static_cast<uint32_t*>(xo), stripe4 ? 1 : 0, rows);
-  return cudaGetLastError();
+  return launch_pdl(prep_block_kernel<S, R>, dim3(grid), dim3(p.groups * p.ntg + 32), R::kSmem, stream,
+                    static_cast<const uint16_t*>(X), T, ldx, static_cast<int>(g.d_in), inv_s, O, jmap,
+                    static_cast<int>(g.k), static_cast<int>(g.k_pad), static_cast<int>(g.kj),
+                    static_cast<int>(g.nblk), p.ntg, aq, sfa, static_cast<uint32_t*>(xo),
+                    stripe4 ? 1 : 0, rows);
 }
 
 bool prep_block_supported(const Geometry& g) {

@@ -1,6 +1,7 @@
 // C-ABI entry points of libw4a4 (declared in include/w4a4.h): argument
 // validation, workspace layout and kernel launches.  No entry point
 // allocates device memory.
+#include <cstdlib>
 #include <cstring>
 
 #include "w4a4.h"
@@ -13,6 +14,15 @@ int device_num_sms() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
   return n;
+}
+
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("W4A4_NO_PDL");
+    on = (e != nullptr && strcmp(e, "1") == 0) ? 0 : 1;
+  }
+  return on == 1;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

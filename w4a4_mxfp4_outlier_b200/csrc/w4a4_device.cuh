@@ -122,6 +122,18 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// Programmatic dependent launch.  A kernel launched with the attribute may
+// start (its CTAs take SMs as the previous kernel's CTAs leave) before the
+// previous kernel in the stream has finished; it runs only shared-memory and
+// tensor-memory setup until pdl_wait(), which returns once the grids it
+// depends on have completed and their memory is visible, and touches global
+// memory only after it.  Without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// lets the next kernel in the stream start launching
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // One lane of a converged warp (always the same lane for a full mask).  The
 // single-thread tcgen05 and TMA instructions are issued under it while the
 // rest of the warp stays converged with the issuer: a lone lane running the

@@ -45,6 +45,31 @@ __host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t b, int6
 
 int device_num_sms();
 
+// Launch attributes of a kernel that calls pdl_wait() before its first
+// global-memory access: programmatic dependent launch, so its launch and
+// setup overlap the end of the previous kernel in the stream.
+// W4A4_NO_PDL=1 in the environment turns it off (read once per process).
+bool pdl_enabled();
+inline int pdl_attrs(cudaLaunchAttribute* attr) {
+  if (!pdl_enabled()) return 0;
+  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr->val.programmaticStreamSerializationAllowed = 1;
+  return 1;
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = static_cast<unsigned>(pdl_attrs(attr));
+  cfg.attrs = attr;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_colabsmax(const void* A, int64_t rows, int64_t cols, int64_t lda, float* absmax,
                              int reset, cudaStream_t stream);
 // both matrices in one launch (A1 may have 0 rows; out1 is then unused)

@@ -33,6 +33,11 @@
  *  - Device-side failures (a pipeline wait that runs out, about 2 s) are
  *    recorded in a device error word; w4a4_last_error() reads it.  No kernel
  *    traps.
+ *  - The calibration, prep and GEMM kernels are launched with programmatic
+ *    dependent launch: they may start their on-chip setup while the previous
+ *    kernel in the stream finishes and wait for it before touching memory,
+ *    so stream order holds as usual.  W4A4_NO_PDL=1 in the environment
+ *    launches them plainly (read once per process).
  */
 #ifndef W4A4_H
 #define W4A4_H

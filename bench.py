@@ -291,9 +291,9 @@ class ClockSampler:
 # (gemm.cu then w4a4_device.cuh); reported as null for any other source or
 # workload.
 GEMM_TRAFFIC = {
-    "sha256": "74f3969d5eec1afe049564ddcdb823c37113c39eb14a4580bf65b6de8ce6b578",
+    "sha256": "d128d573ac3fd7cf4f693eb9eef4ff76026aa6009a48c6bcb2f5878b95f3af41",
     "workload": "full",
-    "mid_bytes": {"up": 167202048 + 408370688, "down": 310143744 + 148844288},
+    "mid_bytes": {"up": 169650176 + 408704512, "down": 320878080 + 149832960},
     "scale": 57600 / 16384,
 }
 

@@ -22,7 +22,10 @@ where a step's inputs are under twice the L2 size a 256 MB buffer is written
 between steps, outside each step's own events.  ``e2e`` times the online
 layer through the library's host-buffer call (w4a4_linear_host: upload of X,
 prep, GEMM, download of Y in one call per layer), with the copies inside the
-timed region; the offline half's device time is reported beside it.
+timed region; the offline half's device time is reported beside it.  The
+default line also carries ``context_ffn``: the FFN pair (up, GELU, down) at
+T = 57600, fused against unfused, timed after everything else
+(``--no-ffn-context`` skips it).
 
 ``--gpus N`` runs N ranks, one per GPU: launched without a launcher around it,
 bench.py starts them itself through torch's launcher (rendezvous on
@@ -508,6 +511,9 @@ def run_gpu(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(layers, runs, rows=256, outs=1024)
+    ffn_ctx = None
+    if rank == 0 and args.workload == "full" and not args.no_ffn_context:
+        ffn_ctx = ffn_context(device)
 
     if rank == 0:
         out = {
@@ -540,6 +546,8 @@ def run_gpu(args):
                 "note": "torch.mm bf16 of the same X and W, timed after the timed region "
                         "(5 reps, L2 not flushed); not part of the step"},
         }
+        if ffn_ctx is not None:
+            out["context_ffn"] = ffn_ctx
         print(json.dumps(out), flush=True)
     if active:
         import torch.distributed as dist
@@ -868,27 +876,19 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def run_ffn(args):
-    """The FFN pair at T=57600 ("ffn"; "ffn_mid": T=16384) (Wan2.2 block: 5120 -> 13824, GELU, 13824 -> 5120)
-    with the down layer fed by the up layer's output.  Both layers are
-    calibrated and packed before the timed region; a step is the online
-    forward of one batch: fused (prep, up GEMM whose epilogue writes the down
-    layer's quantised activations, down GEMM) and, timed after it for
-    comparison, unfused (up linear to bf16 Y, GELU, down linear)."""
+def ffn_setup(Lu, Ld, device, rank=0):
+    """Inputs, calibration and packing of the FFN pair (up layer Lu, down
+    layer Ld, the down layer fed by the up layer's output), and the two
+    forwards: fused (prep, up GEMM whose epilogue writes the down layer's
+    quantised activations, down GEMM; returns its launch count) and unfused
+    (up linear to bf16 Y, GELU, down linear).  Returns (fused, unfused, Y of
+    the fused forward, Y of the unfused one)."""
     import torch
 
     import synth
     import w4a4_mxfp4_outlier_b200 as w4
     from w4a4_mxfp4_outlier_b200 import ffn
 
-    world, rank, local = dist_env()
-    check_device(local)
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    active = dist_init("nccl", world, rank)
-    Lu, Ld = synth.FULL_UP.with_(seed=1000 * rank), synth.FULL_DOWN
-    if args.workload == "ffn_mid":            # the same pair at T=16384 (profiling size)
-        Lu = synth.MID_UP.with_(seed=1000 * rank)
     T, d_model, d_ff = Lu.T, Lu.d_in, Lu.d_out
     X, W_up = synth.gen_layer(Lu, device)
     W_down = synth.gen_w(Ld.w, Ld.d_out, Ld.d_in, seed=Ld.seed + 1 + 1000 * rank, device=device)
@@ -900,7 +900,6 @@ def run_ffn(args):
     Yu = torch.empty((T, d_ff), dtype=torch.bfloat16, device=device)
     H = torch.empty((T, d_ff), dtype=torch.bfloat16, device=device)
     Y2 = torch.empty_like(Y)
-    mk = lambda: torch.cuda.Event(enable_timing=True)
 
     def fused(ev=None):
         if ev: ev[0].record()
@@ -916,6 +915,74 @@ def run_ffn(args):
         w4.linear(X, f.up_plain, ws_u, Yu)
         ffn.gelu_bf16(Yu, H)
         w4.linear(H, f.down, ws_d, Y2)
+
+    return fused, unfused, Y, Y2
+
+
+def ffn_context(device, steps=10, warmup=3):
+    """The FFN pair at T=57600 (fused against unfused), timed after the
+    headline line's own measurements as context: the measurement of
+    `--workload ffn`, without its clock sampling and L2 logic (its inputs are
+    larger than L2)."""
+    import torch
+
+    import synth
+    import w4a4_mxfp4_outlier_b200 as w4
+
+    fused, unfused, Y, Y2 = ffn_setup(synth.FULL_UP, synth.FULL_DOWN, device)
+    for _ in range(warmup):
+        fused()
+        unfused()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[mk() for _ in range(4)] for _ in range(steps)]
+    u_evs = [(mk(), mk()) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for k in range(steps):
+        fused(evs[k])
+    for k in range(steps):
+        u_evs[k][0].record()
+        unfused()
+        u_evs[k][1].record()
+    torch.cuda.synchronize()
+    st, bits = w4.last_error()
+    if st != w4.OK:
+        raise RuntimeError(f"device error word {bits:#x} in the FFN context")
+    avg = lambda i, j: sum(e[i].elapsed_time(e[j]) for e in evs) / steps
+    fused_ms = avg(0, 3)
+    unfused_ms = sum(a.elapsed_time(b) for a, b in u_evs) / steps
+    return {"workload": "ffn: T=57600 5120->13824 k=32 alpha=0.6, GELU, 13824->5120 k=64 alpha=0.7, 32x1",
+            "steps": steps, "fused_ms": round(fused_ms, 4),
+            "prep_ms": round(avg(0, 1), 4), "up_gemm_fused_ms": round(avg(1, 2), 4),
+            "down_gemm_ms": round(avg(2, 3), 4), "unfused_ms": round(unfused_ms, 4),
+            "fused_speedup": round(unfused_ms / fused_ms, 3),
+            "outputs_bit_identical": bool(torch.equal(Y.view(torch.int16), Y2.view(torch.int16))),
+            "note": "online FFN forward (packed weights prepared before timing), timed after the "
+                    "headline measurements; bench.py --workload ffn gives the full line"}
+
+
+def run_ffn(args):
+    """The FFN pair at T=57600 ("ffn"; "ffn_mid": T=16384) (Wan2.2 block: 5120 -> 13824, GELU, 13824 -> 5120)
+    with the down layer fed by the up layer's output.  Both layers are
+    calibrated and packed before the timed region; a step is the online
+    forward of one batch: fused (prep, up GEMM whose epilogue writes the down
+    layer's quantised activations, down GEMM) and, timed after it for
+    comparison, unfused (up linear to bf16 Y, GELU, down linear)."""
+    import torch
+
+    import synth
+    import w4a4_mxfp4_outlier_b200 as w4
+
+    world, rank, local = dist_env()
+    check_device(local)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    active = dist_init("nccl", world, rank)
+    Lu, Ld = synth.FULL_UP.with_(seed=1000 * rank), synth.FULL_DOWN
+    if args.workload == "ffn_mid":            # the same pair at T=16384 (profiling size)
+        Lu = synth.MID_UP.with_(seed=1000 * rank)
+    T, d_model, d_ff = Lu.T, Lu.d_in, Lu.d_out
+    fused, unfused, Y, Y2 = ffn_setup(Lu, Ld, device, rank)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
 
     for _ in range(args.warmup):
         fused()
@@ -1024,6 +1091,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ffn-context", action="store_true",
+                    help="skip the FFN pair (fused against unfused) timed after the headline line")
     ap.add_argument("--report", action="store_true",
                     help="one JSON line per workload configuration (tiny, ffn0, ffn2, the two "
                          "full layers, every sweep point) instead of the headline line")

@@ -334,6 +334,39 @@ def test_tile_widths_give_the_same_bits(tmp_path):
         assert np.array_equal(Y.view(torch.int16).cpu().numpy(), y256), L.name
 
 
+def test_empty_token_batch_is_a_no_op():
+    """T = 0 through every online call and the single-matrix calibration:
+    OK, nothing enqueued that touches memory, and the buffers (filled with a
+    sentinel) unchanged; the next call on the same buffers is still right."""
+    L = RAGGED
+    X, W, pw = _calibrate(L)
+    X0 = X[:0]
+    ws = torch.full((w4.workspace_size(L.T, L.d_in, L.d_out, L.k),), 0x5A, dtype=torch.uint8,
+                    device="cuda")
+    Y = torch.full((L.T, L.d_out), 3.0, dtype=torch.bfloat16, device="cuda")
+    act = w4.alloc_act(L.T, pw)
+    for t in (act.aq, act.sfa):
+        t.fill_(0x5A)
+    act.xo.fill_(3.0)
+    snap = [t.clone() for t in (ws, Y, act.aq, act.sfa, act.xo)]
+    w4.linear(X0, pw, ws, Y[:0])
+    w4.prep_act(X0, pw, act)
+    w4.gemm_dual(act, 0, pw, Y[:0])
+    w4.linear_noalloc(X0, pw, Y[:0])
+    absmax = pw.act_scale.clone()
+    w4.calib_observe(X0, absmax, reset=False)
+    torch.cuda.synchronize()
+    for a, b in zip(snap, (ws, Y, act.aq, act.sfa, act.xo)):
+        assert torch.equal(a, b)
+    assert torch.equal(absmax, pw.act_scale)
+    st, bits = w4.last_error()
+    assert st == w4.OK, f"device error word {bits:#x}"
+    Y1 = _linear(X, pw, L.T, L.d_out)
+    w4.linear(X, pw, ws, Y)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y1)
+
+
 def test_gemm_matches_linear_and_is_deterministic():
     L = RAGGED
     X, W, pw = _calibrate(L)

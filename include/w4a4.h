@@ -134,8 +134,9 @@ w4a4_status w4a4_calib_observe_layer(const void* X, int64_t T, int64_t ldx, cons
  *   O        = the k columns of largest score, ties to the lower index,
  *              ascending (int32 [k]);  jmap = the other d_in - k columns
  *              ascending (int32 [d_in - k]).
- * Requires 0 < alpha < 1, 0 <= k <= d_in, 1 <= d_in <= 65535.  O may be NULL
- * when k == 0 and jmap may be NULL when k == d_in.
+ * Requires 0 < alpha < 1, 0 <= k <= d_in, d_in >= 1 (else INVALID_ARG);
+ * d_in > 16384 returns UNSUPPORTED_SHAPE.  O may be NULL when k == 0 and
+ * jmap may be NULL when k == d_in.
  * s is defined for finite magnitudes only: if act_scale or w_scale holds an
  * inf or a NaN (calibration data that were not finite), the kernel records it
  * in the device error word -- w4a4_last_error then returns
